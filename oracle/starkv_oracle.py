@@ -75,6 +75,19 @@ def factors_from_svd(U: np.ndarray, s: np.ndarray, V: np.ndarray, r: int):
     return U[:, :r] * s[None, :r], V[:, :r].T.copy()
 
 
+def canonical_signs(A, B):
+    """Fix the sign freedom of each singular pair: row i of B (a right singular vector) is
+    negated, together with column i of A, when its entry of largest magnitude is negative.
+    A @ B is unchanged; the convention gives a drawn latent channel one meaning."""
+    B = np.array(B, dtype=np.float64, copy=True)
+    idx = np.argmax(np.abs(B), axis=1)
+    flip = np.where(B[np.arange(B.shape[0]), idx] < 0, -1.0, 1.0)
+    B *= flip[:, None]
+    if A is not None:
+        A = np.array(A, dtype=np.float64, copy=True) * flip[None, :]
+    return A, B
+
+
 # ======================================================================================
 # [S2] joint and head-wise decompositions
 # ======================================================================================
@@ -440,3 +453,56 @@ def decode_attention(q, C_k, C_v, B_k, B_v, theta: float, n_kv_heads: int, heads
 def project(x, A) -> np.ndarray:
     """Latent write of new tokens: c = x A, with A = [A_k | A_v,0 | A_v,1 | ...] [AB]."""
     return np.asarray(x, np.float64) @ np.asarray(A, np.float64)
+
+
+# ======================================================================================
+# the same quantiser over many tokens at once (NumPy vector form of quantize_latent /
+# dequantize_latent; pinned against the per-token definitions by the tests)
+# ======================================================================================
+def _quantize_block(C: np.ndarray, bits: int):
+    """C: (n, k) fp32 group members (k <= 32).  Returns fp16 scales (n,), codes (n, k)."""
+    qmax = np.float32((1 << (bits - 1)) - 1)
+    amax = np.max(np.abs(C), axis=1) if C.shape[1] else np.zeros(C.shape[0], np.float32)
+    with np.errstate(over="ignore"):
+        s16 = (amax.astype(np.float32) / qmax).astype(np.float16)
+    s16 = np.where(np.isfinite(s16), s16, np.float16(65504.0)).astype(np.float16)
+    s = s16.astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = C / s[:, None]
+    q = np.clip(np.rint(r), -qmax, qmax)
+    q = np.where(s[:, None] == 0, 0, q)
+    return s16, q.astype(np.int8)
+
+
+def quantize_rows(C, r: int):
+    """quantize_latent for every row of C (n, r) fp32: (q8 (n, n8), q4 (n, n4), scales (n, ng))."""
+    C = np.asarray(C, dtype=np.float32)
+    sp = mixed_split(r)
+    n8, n4 = sp["n8"], sp["n4"]
+    scales, q8, q4 = [], [], []
+    for gi in range(sp["g8"]):
+        s, q = _quantize_block(C[:, gi * GROUP:min((gi + 1) * GROUP, n8)], 8)
+        scales.append(s)
+        q8.append(q)
+    for gi in range(sp["g4"]):
+        s, q = _quantize_block(C[:, n8 + gi * GROUP:n8 + min((gi + 1) * GROUP, n4)], 4)
+        scales.append(s)
+        q4.append(q)
+    n = C.shape[0]
+    q8 = np.concatenate(q8, axis=1) if q8 else np.zeros((n, 0), np.int8)
+    q4 = np.concatenate(q4, axis=1) if q4 else np.zeros((n, 0), np.int8)
+    return q8, q4, np.stack(scales, axis=1)
+
+
+def dequantize_rows(q8, q4, scales, r: int) -> np.ndarray:
+    sp = mixed_split(r)
+    s8 = np.repeat(scales[:, :sp["g8"]].astype(np.float64), GROUP, axis=1)[:, :sp["n8"]]
+    s4 = np.repeat(scales[:, sp["g8"]:].astype(np.float64), GROUP, axis=1)[:, :sp["n4"]]
+    return np.concatenate([s8 * q8, s4 * q4], axis=1)
+
+
+def stored_rows(C, r: int, fmt: str) -> np.ndarray:
+    """Stored value (fp64) of every row of C (n, r) fp32 in format ``fmt``."""
+    if fmt == MIXED:
+        return dequantize_rows(*quantize_rows(C, r), r)
+    return store_latents(C, fmt)

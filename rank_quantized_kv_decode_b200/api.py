@@ -1,0 +1,156 @@
+"""Python binding of the C ABI.  Argument marshalling only: every step of the hot path runs
+in the CUDA library; PyTorch supplies device memory and the stream.
+
+Names mirror include/starkv.h (``starkv_append`` -> ``append`` ...).  Tensors must be
+contiguous CUDA tensors on the current device; dtypes follow the header.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib as L
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def make_config(n_q_heads: int, n_kv_heads: int, head_dim: int, d_model: int, key_rank: int,
+                value_ranks, fmt: str, rope_theta: float, page_tokens: int = 64) -> L.Config:
+    c = L.Config()
+    c.n_q_heads, c.n_kv_heads, c.head_dim, c.d_model = n_q_heads, n_kv_heads, head_dim, d_model
+    c.key_rank = key_rank
+    if len(value_ranks) != n_kv_heads:
+        raise ValueError("one value rank per KV head")
+    for g, r in enumerate(value_ranks):
+        c.value_rank[g] = int(r)
+    c.fmt = L.FMT[fmt]
+    c.page_tokens = page_tokens
+    c.rope_theta = float(rope_theta)
+    return c
+
+
+def layout_init(cfg: L.Config) -> L.Layout:
+    lay = L.Layout()
+    L.check(L.load().starkv_layout_init(ctypes.byref(cfg), ctypes.byref(lay)), "starkv_layout_init")
+    return lay
+
+
+def alloc(lay: L.Layout, num_pages: int, batch: int, max_pages: int,
+          max_append_tokens: int) -> L.Sizes:
+    s = L.Sizes()
+    L.check(L.load().starkv_alloc(ctypes.byref(lay), num_pages, batch, max_pages,
+                                  max_append_tokens, ctypes.byref(s)), "starkv_alloc")
+    return s
+
+
+def rope_init(lay: L.Layout, max_pages: int, table: torch.Tensor, stream=None) -> None:
+    L.check(L.load().starkv_rope_init(ctypes.byref(lay), max_pages, _ptr(table),
+                                      table.numel() * table.element_size(), _stream(stream)),
+            "starkv_rope_init")
+
+
+def quant_pack(lay, latents, tok_seq, tok_pos, block_table, cache, status, stream=None) -> None:
+    n_tok = latents.shape[0]
+    L.check(L.load().starkv_quant_pack(
+        ctypes.byref(lay), _ptr(latents), n_tok, _ptr(tok_seq), _ptr(tok_pos), _ptr(block_table),
+        block_table.shape[1], block_table.shape[0], _ptr(cache),
+        cache.numel() * cache.element_size() // lay.page_bytes, _ptr(status), _stream(stream)),
+        "starkv_quant_pack")
+
+
+def append(lay, x, A_t, tok_seq, tok_pos, block_table, cache, workspace, status,
+           latents_out=None, stream=None) -> None:
+    L.check(L.load().starkv_append(
+        ctypes.byref(lay), _ptr(x), x.shape[0], _ptr(A_t), _ptr(tok_seq), _ptr(tok_pos),
+        _ptr(block_table), block_table.shape[1], block_table.shape[0], _ptr(cache),
+        cache.numel() * cache.element_size() // lay.page_bytes, _ptr(latents_out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)), "starkv_append")
+
+
+def dequant(lay, cache, tok_seq, tok_pos, block_table, latents_out, status, stream=None) -> None:
+    L.check(L.load().starkv_dequant(
+        ctypes.byref(lay), _ptr(cache), cache.numel() * cache.element_size() // lay.page_bytes,
+        _ptr(tok_seq), _ptr(tok_pos), tok_seq.shape[0], _ptr(block_table), block_table.shape[1],
+        block_table.shape[0], _ptr(latents_out), _ptr(status), _stream(stream)), "starkv_dequant")
+
+
+def decode_attention(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rope_table, out, workspace,
+                     status, max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
+                     stream=None) -> None:
+    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms)
+    L.check(L.load().starkv_decode_attention(
+        ctypes.byref(lay), _ptr(q), _ptr(cache),
+        cache.numel() * cache.element_size() // lay.page_bytes, _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], _ptr(Bk_t), _ptr(Bv),
+        _ptr(rope_table), rope_table.numel() * rope_table.element_size(), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), ctypes.byref(opts),
+        _ptr(status), _stream(stream)), "starkv_decode_attention")
+
+
+def decode_partials(lay, q, cache, block_table, seq_lens, Bk_t, rope_table, workspace, status,
+                    max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
+                    stream=None) -> None:
+    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms)
+    L.check(L.load().starkv_decode_partials(
+        ctypes.byref(lay), _ptr(q), _ptr(cache),
+        cache.numel() * cache.element_size() // lay.page_bytes, _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], _ptr(Bk_t), _ptr(rope_table),
+        rope_table.numel() * rope_table.element_size(), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), ctypes.byref(opts), _ptr(status),
+        _stream(stream)), "starkv_decode_partials")
+
+
+def decode_combine(lay, seq_lens, max_pages: int, Bv, workspace, out, stream=None) -> None:
+    L.check(L.load().starkv_decode_combine(
+        ctypes.byref(lay), _ptr(seq_lens), seq_lens.shape[0], max_pages, _ptr(Bv),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
+        _stream(stream)), "starkv_decode_combine")
+
+
+def _bytes(n: int, device) -> torch.Tensor:
+    # 256-byte aligned raw buffer (the caching allocator aligns blocks to 512 bytes)
+    return torch.empty(max(int(n), 16), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class LatentCache:
+    """Caller-side buffers of one layer's compressed cache: the page pool, the RoPE table and
+    the workspaces, sized by ``starkv_alloc``.  Plain device memory owned by PyTorch."""
+
+    layout: L.Layout
+    num_pages: int
+    batch: int
+    max_pages: int
+    max_append_tokens: int
+    cache: torch.Tensor
+    rope: torch.Tensor
+    decode_ws: torch.Tensor
+    append_ws: torch.Tensor
+    status: torch.Tensor
+
+    @classmethod
+    def create(cls, lay: L.Layout, num_pages: int, batch: int, max_pages: int,
+               max_append_tokens: int, device="cuda") -> "LatentCache":
+        s = alloc(lay, num_pages, batch, max_pages, max_append_tokens)
+        c = cls(lay, num_pages, batch, max_pages, max_append_tokens,
+                _bytes(s.cache_bytes, device), _bytes(s.rope_table_bytes, device),
+                _bytes(s.decode_workspace_bytes, device), _bytes(s.append_workspace_bytes, device),
+                torch.zeros(1, dtype=torch.int32, device=device))
+        rope_init(lay, max_pages, c.rope)
+        return c

@@ -1,0 +1,651 @@
+// Decode attention read straight from the latent cache (sm_100a).
+//
+// Split kernel (persistent, warp-specialised, one CTA per SM).  A work unit is one
+// 128-token tile (two 64-token pages) of one sequence and a range of 256-column chunks of
+// the reconstructed keys (2 KV heads of d=128, or 4 of d=64):
+//   warp 0      TMA producer: latent k-blocks of the two pages (f32/bf16) and B_k^T k-blocks
+//   warp 1      tcgen05 issuer: K_chunk = C_k(128 x r_k) * B_k(r_k x 256) into TMEM (fp32),
+//               double-buffered accumulators (2 x 256 columns)
+//   warp 2      bulk-copy producer of the value latents of the chunk's heads (both pages)
+//   warps 4-11  two epilogue warpgroups, one per 128 TMEM columns: thread = token row;
+//               RoPE on the key row, scores against the rotated queries of the GQA group,
+//               tile-local softmax (max, sum), latent P.C_v, one partial per query head
+//   warps 12-15 (int8/int4 format) dequantisers: codes * fp16 scale -> fp16 operand tile in
+//               the 128-byte-swizzled layout the tensor core reads
+// The pages' point that joint key latents cost h x more to reconstruct (STAR-KV technical
+// summary, Methodology §2 "Hybrid Decomposition Strategy") is why the reconstruction runs
+// on the tensor cores: it is a dense (tokens x r_k) x (r_k x H_kv*d) contraction.
+//
+// Combine kernel: log-sum-exp merge of the per-tile partials of each (sequence, query head),
+// then the up-projection o_h = a_h B_v,g.
+#include "internal.cuh"
+
+namespace starkv {
+
+namespace {
+
+constexpr int FMT_F32 = STARKV_FMT_F32;
+constexpr int FMT_BF16 = STARKV_FMT_BF16;
+constexpr int FMT_MIXED = STARKV_FMT_MIXED;
+
+struct Unit {
+  int b, tile, c0, c1, L, nvalid;
+  int page0, page1;  // physical pages of the tile's two halves, -1 if absent or invalid
+  __device__ __forceinline__ int page(int half) const { return half ? page1 : page0; }
+};
+
+// Same answer in every role: the pipelines of all warps walk the same unit sequence.
+__device__ __forceinline__ bool get_unit(const DecodeParams& p, int u, Unit& U, bool flag) {
+  const int rg = u % p.n_ranges;
+  const int rest = u / p.n_ranges;
+  U.b = rest % p.batch;
+  U.tile = rest / p.batch;
+  int L = p.seq_lens[U.b];
+  const int cap = p.max_pages * kPage;
+  if (L > cap || L < 0) {
+    if (flag && p.status) atomicOr(p.status, STARKV_DEV_BOUNDS);
+    L = L < 0 ? 0 : cap;
+  }
+  U.L = L;
+  if (U.tile * kTile >= L) return false;
+  U.c0 = rg * p.cpr;
+  U.c1 = min(U.c0 + p.cpr, p.n_chunks);
+  if (U.c0 >= U.c1) return false;
+  U.nvalid = min(kTile, L - U.tile * kTile);
+  int pgs[2];
+#pragma unroll
+  for (int pp = 0; pp < 2; ++pp) {
+    int pg = -1;
+    if (pp * kPage < U.nvalid) {
+      pg = p.block_table[(long long)U.b * p.max_pages + U.tile * 2 + pp];
+      if (pg < 0 || pg >= p.num_pages) {
+        if (flag && p.status) atomicOr(p.status, STARKV_DEV_BOUNDS);
+        pg = -1;
+      }
+    }
+    pgs[pp] = pg;
+  }
+  U.page0 = pgs[0];
+  U.page1 = pgs[1];
+  return true;
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+  return true;
+}
+
+template <int FMT>
+struct Fmt {
+  static constexpr bool kTmaA = FMT != FMT_MIXED;
+  static constexpr int kKind = FMT == FMT_F32 ? 1 : 0;
+  static constexpr int kElem = FMT == FMT_F32 ? 4 : 2;
+  static constexpr int kKElems = kKBytes / kElem;  // elements per k-block
+  static constexpr int kWarps = kTmaA ? 12 : 16;
+};
+
+// Stored value of value-latent channel i of token row ``row`` (0..63) in a staged page slot.
+template <int FMT>
+__device__ __forceinline__ float vload(const uint8_t* slot, const LatDesc& vd, int vbase, int row,
+                                       int i) {
+  if constexpr (FMT == FMT_F32) {
+    return reinterpret_cast<const float*>(slot + vd.off0 - vbase)[row * vd.rank + i];
+  } else if constexpr (FMT == FMT_BF16) {
+    return __bfloat162float(
+        reinterpret_cast<const __nv_bfloat16*>(slot + vd.off0 - vbase)[row * vd.rank + i]);
+  } else {
+    const __half* sc = reinterpret_cast<const __half*>(slot + vd.off2 - vbase) + row * vd.ng;
+    if (i < vd.n8) {
+      const int8_t q = reinterpret_cast<const int8_t*>(slot + vd.off0 - vbase)[row * vd.n8 + i];
+      return __half2float(sc[i >> 5]) * static_cast<float>(q);
+    }
+    const int j = i - vd.n8;
+    const uint8_t byte = (slot + vd.off1 - vbase)[row * vd.nb4 + (j >> 1)];
+    const int nib = (j & 1) ? (byte >> 4) : (byte & 15);
+    return __half2float(sc[vd.g8 + (j >> 5)]) * static_cast<float>((nib ^ 8) - 8);
+  }
+}
+
+// 8 consecutive key-latent channels [k0, k0+8) of one token as fp16 (scale * code, rounded
+// to nearest), packed for one 16-byte store.  ``base`` is the page.
+__device__ __forceinline__ float key_code_value(const uint8_t* base, const LatDesc& kd, int prow,
+                                                int k) {
+  const __half* sc = reinterpret_cast<const __half*>(base + kd.off2) + prow * kd.ng;
+  if (k < kd.n8) {
+    const int8_t q = reinterpret_cast<const int8_t*>(base + kd.off0)[prow * kd.n8 + k];
+    return __half2float(sc[k >> 5]) * static_cast<float>(q);
+  }
+  const int j = k - kd.n8;
+  const uint8_t byte = (base + kd.off1)[prow * kd.nb4 + (j >> 1)];
+  const int nib = (j & 1) ? (byte >> 4) : (byte & 15);
+  return __half2float(sc[kd.g8 + (j >> 5)]) * static_cast<float>((nib ^ 8) - 8);
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint4 dequant8(const DecodeParams& p, const Unit& U, int r, int k0) {
+  uint4 z = make_uint4(0, 0, 0, 0);
+  const int pp = r >> 6, prow = r & 63;
+  const int pg = U.page(pp);
+  const LatDesc& kd = p.key;
+  if (pg < 0 || r >= U.nvalid || k0 >= kd.rank) return z;
+  const uint8_t* base = p.cache + (long long)pg * p.page_bytes;
+  float v[8];
+  if (k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(base + kd.off0 + prow * kd.n8 + k0);
+    const float s = __half2float(reinterpret_cast<const __half*>(base + kd.off2)[prow * kd.ng + (k0 >> 5)]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[e] = s * static_cast<float>(static_cast<int8_t>((raw.x >> (8 * e)) & 0xFF));
+      v[4 + e] = s * static_cast<float>(static_cast<int8_t>((raw.y >> (8 * e)) & 0xFF));
+    }
+  } else if (k0 >= kd.n8 && ((k0 - kd.n8) & 7) == 0 && k0 + 8 <= kd.rank && (kd.nb4 & 3) == 0) {
+    const int j0 = k0 - kd.n8;
+    const uint32_t raw = *reinterpret_cast<const uint32_t*>(base + kd.off1 + prow * kd.nb4 + (j0 >> 1));
+    const float s =
+        __half2float(reinterpret_cast<const __half*>(base + kd.off2)[prow * kd.ng + kd.g8 + (j0 >> 5)]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int nib = (raw >> (4 * e)) & 15;
+      v[e] = s * static_cast<float>((nib ^ 8) - 8);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int k = k0 + e;
+      v[e] = k < kd.rank ? key_code_value(base, kd, prow, k) : 0.f;
+    }
+  }
+  z.x = pack_h2(v[0], v[1]);
+  z.y = pack_h2(v[2], v[3]);
+  z.z = pack_h2(v[4], v[5]);
+  z.w = pack_h2(v[6], v[7]);
+  return z;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int FMT>
+__device__ __forceinline__ float qload(const void* q, long long idx) {
+  if constexpr (FMT == FMT_F32) return reinterpret_cast<const float*>(q)[idx];
+  else return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[idx]);
+}
+
+}  // namespace
+
+template <int FMT, int HD, int G>
+__global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
+    decode_split_kernel(const __grid_constant__ DecodeParams p,
+                        const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB) {
+  using F = Fmt<FMT>;
+  constexpr int HPW = 128 / HD;  // KV heads per epilogue warpgroup
+  constexpr int QPW = HPW * G;   // query heads per epilogue warpgroup
+  constexpr int HALF = HD / 2;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.stages, NVB = p.nvb;
+  const uint32_t bstage = static_cast<uint32_t>(p.NC) * kKBytes;
+
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + p.off_b;
+  uint8_t* sV = smem + p.off_v;
+  float* sQ = reinterpret_cast<float*>(smem + p.off_q);    // [2][QPW][HD]
+  float* sP = reinterpret_cast<float*>(smem + p.off_p);    // [2][QPW][128]
+  float* sRed = reinterpret_cast<float*>(smem + p.off_red);  // [2][2][QPW][4]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  const int B_FULL = 0, B_EMPTY = S, B_ACCF = 2 * S, B_ACCE = 2 * S + 2, B_VF = 2 * S + 4,
+            B_VE = 2 * S + 4 + NVB, B_TD = 2 * S + 4 + 2 * NVB;
+  // misc: [0] TMEM base, [1] abort flag, [2..3] per-warpgroup stop snapshots
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + B_TD + 1);
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar(B_FULL + s), F::kTmaA ? 1 : 5);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar(B_ACCF + a), 1);
+      mbar_init(bar(B_ACCE + a), 8);
+    }
+    for (int v = 0; v < NVB; ++v) {
+      mbar_init(bar(B_VF + v), 1);
+      mbar_init(bar(B_VE + v), 8);
+    }
+    mbar_init(bar(B_TD), 1);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmB);
+    if constexpr (F::kTmaA) prefetch_tmap(&tmA);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(misc), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  WaitCtl wc{reinterpret_cast<volatile int*>(misc + 1), p.status, p.timeout_ns};
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, last_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        Unit U;
+        if (!get_unit(p, u, U, true)) continue;
+        for (int c = U.c0; ok && c < U.c1; ++c) {
+          for (int kb = 0; kb < p.kb_count; ++kb) {
+            if (!wait_bounded(bar(B_EMPTY + stage), phase ^ 1u, wc)) { ok = false; break; }
+            uint32_t bytes = bstage;
+            if constexpr (F::kTmaA)
+              bytes += (U.page0 >= 0 ? 8192u : 0u) + (U.page1 >= 0 ? 8192u : 0u);
+            const uint32_t fb = bar(B_FULL + stage);
+            mbar_arrive_expect_tx(fb, bytes);
+            if constexpr (F::kTmaA) {
+              const uint32_t da = smem_u32(sA + stage * kAStage);
+              if (U.page0 >= 0) tma_load_3d(da, &tmA, fb, kb * F::kKElems, 0, U.page0);
+              if (U.page1 >= 0) tma_load_3d(da + 8192, &tmA, fb, kb * F::kKElems, 0, U.page1);
+            }
+            tma_load_2d(smem_u32(sB + stage * bstage), &tmB, fb, kb * F::kKElems, c * p.NC);
+            issued |= 1u << stage;
+            last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == S) { stage = 0; phase ^= 1u; }
+          }
+        }
+      }
+      // every copy this thread started has landed before the CTA may exit
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) wait_drain(bar(B_FULL + s), (last_phase >> s) & 1u, p.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0, ab = 0;
+      uint32_t phase = 0, aph = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        Unit U;
+        if (!get_unit(p, u, U, false)) continue;
+        for (int c = U.c0; ok && c < U.c1; ++c) {
+          if (!wait_bounded(bar(B_ACCE + ab), aph ^ 1u, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * 256);
+          for (int kb = 0; kb < p.kb_count; ++kb) {
+            if (!wait_bounded(bar(B_FULL + stage), phase, wc)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t da = desc_sw128(smem_u32(sA + stage * kAStage));
+            const uint64_t db = desc_sw128(smem_u32(sB + stage * bstage));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma<F::kKind>(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
+            umma_commit(bar(B_EMPTY + stage));
+            if (++stage == S) { stage = 0; phase ^= 1u; }
+          }
+          if (!ok) break;
+          umma_commit(bar(B_ACCF + ab));
+          ab ^= 1;
+          if (ab == 0) aph ^= 1u;
+        }
+      }
+      umma_commit(bar(B_TD));
+      wait_drain(bar(B_TD), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ---------------------------------------------------------------- value-latent producer
+    if (lane == 0) {
+      int vs = 0;
+      uint32_t vph = 0, issued = 0, last_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        Unit U;
+        if (!get_unit(p, u, U, false)) continue;
+        for (int c = U.c0; c < U.c1; ++c) {
+          if (!wait_bounded(bar(B_VE + vs), vph ^ 1u, wc)) { ok = false; break; }
+          const uint32_t nbytes = static_cast<uint32_t>(p.vchunk_bytes[c]);
+          const uint32_t fb = bar(B_VF + vs);
+          mbar_arrive_expect_tx(fb, nbytes * ((U.page0 >= 0) + (U.page1 >= 0)));
+          for (int pp = 0; pp < 2; ++pp) {
+            const int pg = U.page(pp);
+            if (pg < 0) continue;
+            const uint8_t* src = p.cache + (long long)pg * p.page_bytes + p.vchunk_off[c];
+            bulk_g2s(smem_u32(sV + (vs * 2 + pp) * p.vslot), src, nbytes, fb);
+          }
+          issued |= 1u << vs;
+          last_phase = (last_phase & ~(1u << vs)) | (vph << vs);
+          if (++vs == NVB) { vs = 0; vph ^= 1u; }
+        }
+      }
+      for (int v = 0; v < NVB; ++v)
+        if (issued & (1u << v)) wait_drain(bar(B_VF + v), (last_phase >> v) & 1u, p.timeout_ns);
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------------------------------------------------------- epilogue warpgroups
+    const int wg = (warp - 4) >> 2;
+    const int quad = warp & 3;          // TMEM lane quadrant of this warp
+    const int row = quad * 32 + lane;   // token row in the tile == thread index in the WG
+    const float2* fine = p.rope;
+    const float2* basetab = p.rope + kTile * HALF;
+    float* q_s = sQ + wg * QPW * HD;
+    float* p_s = sP + wg * QPW * kTile;
+    float* red = sRed + wg * 2 * QPW * 4;
+    int* s_stop = reinterpret_cast<int*>(misc + 2);  // [2] per-warpgroup snapshot of abort
+    int ab = 0, vs = 0;
+    uint32_t aph = 0, vph = 0;
+    // Control flow of a warpgroup only changes on a snapshot every thread reads after a
+    // named barrier, so no thread can leave while the others wait at a barrier.
+    bool stop = false;
+    for (int u = blockIdx.x; !stop && u < p.total_units; u += gridDim.x) {
+      Unit U;
+      if (!get_unit(p, u, U, false)) continue;
+      const int T = U.L - 1;  // position of the decode query
+      const bool rv = row < U.nvalid && U.page(row >> 6) >= 0;
+      const float2* fine_r = fine + row * HALF;
+      const float2* base_t = basetab + U.tile * HALF;
+      for (int c = U.c0; c < U.c1; ++c) {
+        const int g_first = c * (p.NC / HD) + wg * HPW;
+        // (1) rotated, scaled queries of this warpgroup's heads
+        for (int idx = row; idx < QPW * HALF; idx += 128) {
+          const int hq = idx / HALF, j = idx % HALF;
+          const int g = g_first + hq / G;
+          if (g >= p.Hkv) continue;
+          const int h = g * G + hq % G;
+          const long long qb = ((long long)U.b * p.H + h) * HD;
+          const float x0 = qload<FMT>(p.q, qb + j), x1 = qload<FMT>(p.q, qb + j + HALF);
+          const float2 bs = basetab[(T >> 7) * HALF + j], f = fine[(T & 127) * HALF + j];
+          const float cs = bs.x * f.x - bs.y * f.y, sn = bs.y * f.x + bs.x * f.y;
+          q_s[hq * HD + j] = (x0 * cs - x1 * sn) * p.qscale;
+          q_s[hq * HD + j + HALF] = (x1 * cs + x0 * sn) * p.qscale;
+        }
+        named_bar(1 + wg, 128);
+        // (2) accumulator of this chunk (on a timeout the data is garbage and the snapshot
+        // below ends the loop)
+        wait_bounded(bar(B_ACCF + ab), aph, wc);
+        tc_fence_after();
+        // (3) RoPE on the reconstructed key row, scores of the GQA group
+        float sc[QPW];
+#pragma unroll
+        for (int hs = 0; hs < HPW; ++hs) {
+          float acc[G];
+#pragma unroll
+          for (int gq = 0; gq < G; ++gq) acc[gq] = 0.f;
+          if (g_first + hs < p.Hkv) {
+            const uint32_t taddr = tmem + static_cast<uint32_t>(ab * 256 + wg * 128 + hs * HD) +
+                                   (static_cast<uint32_t>(quad * 32) << 16);
+#pragma unroll 1
+            for (int jj = 0; jj < HALF; jj += 32) {
+              float klo[32], khi[32];
+              tmem_ld32x2_wait(taddr + jj, taddr + HALF + jj, klo, khi);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float2 f = fine_r[jj + j], bs = base_t[jj + j];
+                const float cs = bs.x * f.x - bs.y * f.y, sn = bs.y * f.x + bs.x * f.y;
+                const float k0 = klo[j] * cs - khi[j] * sn;
+                const float k1 = khi[j] * cs + klo[j] * sn;
+#pragma unroll
+                for (int gq = 0; gq < G; ++gq) {
+                  const float* qq = q_s + (hs * G + gq) * HD + jj + j;
+                  acc[gq] = fmaf(k0, qq[0], fmaf(k1, qq[HALF], acc[gq]));
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int gq = 0; gq < G; ++gq) sc[hs * G + gq] = rv ? acc[gq] : -INFINITY;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_ACCE + ab));
+        ab ^= 1;
+        if (ab == 0) aph ^= 1u;
+        // (4) tile-local softmax statistics (log2 domain: scores carry log2(e)/sqrt(d))
+#pragma unroll
+        for (int hq = 0; hq < QPW; ++hq) {
+          const float m = warp_max(sc[hq]);
+          if (lane == 0) red[hq * 4 + quad] = m;
+        }
+        if (row == 0) s_stop[wg] = *wc.abort_flag;
+        named_bar(1 + wg, 128);
+        if (s_stop[wg]) { stop = true; break; }
+        float mx[QPW];
+#pragma unroll
+        for (int hq = 0; hq < QPW; ++hq) {
+          mx[hq] = fmaxf(fmaxf(red[hq * 4 + 0], red[hq * 4 + 1]), fmaxf(red[hq * 4 + 2], red[hq * 4 + 3]));
+          const float pe = rv ? exp2f(sc[hq] - mx[hq]) : 0.f;
+          p_s[hq * kTile + row] = pe;
+          const float s = warp_sum(pe);
+          if (lane == 0) red[QPW * 4 + hq * 4 + quad] = s;
+        }
+        named_bar(1 + wg, 128);
+        // (5) value latents of this chunk
+        wait_bounded(bar(B_VF + vs), vph, wc);
+        // (6) latent P.C_v and the partial record of each query head
+        const uint8_t* vslot0 = sV + (vs * 2) * p.vslot;
+        const int vbase = p.vchunk_off[c];
+#pragma unroll
+        for (int hs = 0; hs < HPW; ++hs) {
+          const int g = g_first + hs;
+          if (g >= p.Hkv) continue;
+          const LatDesc& vd = p.vh[g];
+          if (row < vd.rank) {
+            float a[G];
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq) a[gq] = 0.f;
+            for (int pp = 0; pp < 2; ++pp) {
+              if (U.page(pp) < 0) continue;
+              const uint8_t* slot = vslot0 + pp * p.vslot;
+              const int t1 = min(kPage, U.nvalid - pp * kPage);
+#pragma unroll 4
+              for (int t = 0; t < t1; ++t) {
+                const float cv = vload<FMT>(slot, vd, vbase, t, row);
+#pragma unroll
+                for (int gq = 0; gq < G; ++gq)
+                  a[gq] = fmaf(p_s[(hs * G + gq) * kTile + pp * kPage + t], cv, a[gq]);
+              }
+            }
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq) {
+              const int h = g * G + gq;
+              float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
+              rec[2 + row] = a[gq];
+            }
+          }
+          if (row == 0) {
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq) {
+              const int h = g * G + gq;
+              float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
+              const int hq = hs * G + gq;
+              rec[0] = mx[hq];
+              rec[1] = red[QPW * 4 + hq * 4 + 0] + red[QPW * 4 + hq * 4 + 1] +
+                       red[QPW * 4 + hq * 4 + 2] + red[QPW * 4 + hq * 4 + 3];
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_VE + vs));
+        if (++vs == NVB) { vs = 0; vph ^= 1u; }
+      }
+    }
+  } else if (warp >= 12) {
+    // ---------------------------------------------------------------- dequantisers (int8/int4)
+    if constexpr (!F::kTmaA) {
+      const int tid = (warp - 12) * 32 + lane;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        Unit U;
+        if (!get_unit(p, u, U, false)) continue;
+        for (int c = U.c0; ok && c < U.c1; ++c) {
+          for (int kb = 0; kb < p.kb_count; ++kb) {
+            // warp-uniform decision (the __syncwarp below needs every lane)
+            if (!__all_sync(0xffffffffu, wait_bounded(bar(B_EMPTY + stage), phase ^ 1u, wc))) {
+              ok = false;
+              break;
+            }
+            uint8_t* dst = sA + stage * kAStage;
+            const int ch = tid & 7;
+#pragma unroll 2
+            for (int it = 0; it < 8; ++it) {
+              const int r = it * 16 + (tid >> 3);
+              const uint4 v = dequant8(p, U, r, kb * 64 + ch * 8);
+              *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch)) = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_FULL + stage));
+            if (++stage == S) { stage = 0; phase ^= 1u; }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// --------------------------------------------------------------------------- combine
+// One CTA per (sequence, query head): merge the tile partials (m in log2 units, l, a[r]),
+// normalise, then o = a B_v,g.
+__global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
+  const int bh = blockIdx.x;
+  const int b = bh / p.H, h = bh % p.H, g = h / p.G;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ float s_m[4];
+  __shared__ float s_acc[4][129];
+  __shared__ float s_a[128];
+  const LatDesc& vd = p.vh[g];
+  const int r = vd.rank;
+  float* outp = p.out + ((long long)b * p.H + h) * p.d;
+  int L = p.seq_lens[b];
+  L = max(0, min(L, p.max_pages * kPage));
+  if (L == 0) {
+    for (int c = tid; c < p.d; c += 128) outp[c] = 0.f;
+    return;
+  }
+  const int T = (L + kTile - 1) / kTile;
+  const float* recs = p.ws + ((long long)b * p.H + h) * p.tiles_max * p.rec;
+  float m = -INFINITY;
+  for (int t = tid; t < T; t += 128) {
+    const float* rc = recs + (long long)t * p.rec;
+    if (rc[1] > 0.f) m = fmaxf(m, rc[0]);
+  }
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  if (lane == 0) s_m[warp] = m;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(s_m[0], s_m[1]), fmaxf(s_m[2], s_m[3]));
+  // each warp takes every 4th tile; lanes cover the latent channels
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float lsum = 0.f;
+  for (int t = warp; t < T; t += 4) {
+    const float* rc = recs + (long long)t * p.rec;
+    const float lt = rc[1];
+    if (!(lt > 0.f)) continue;
+    const float w = exp2f(rc[0] - M);
+    lsum += lt * w;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = lane + 32 * k;
+      if (i < r) acc[k] = fmaf(rc[2 + i], w, acc[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) s_acc[warp][lane + 32 * k] = acc[k];
+  if (lane == 0) s_acc[warp][128] = lsum;
+  __syncthreads();
+  const float l = s_acc[0][128] + s_acc[1][128] + s_acc[2][128] + s_acc[3][128];
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  if (tid < r) s_a[tid] = (s_acc[0][tid] + s_acc[1][tid] + s_acc[2][tid] + s_acc[3][tid]) * inv;
+  __syncthreads();
+  const float* Bv = p.Bv + (long long)(vd.col - p.key_rank_cols) * p.d;
+  for (int c = tid; c < p.d; c += 128) {
+    float o = 0.f;
+    for (int i = 0; i < r; ++i) o = fmaf(s_a[i], Bv[(long long)i * p.d + c], o);
+    outp[c] = o;
+  }
+}
+
+// --------------------------------------------------------------------------- launchers
+template <int FMT, int HD, int G>
+static cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tmA,
+                              const CUtensorMap& tmB, int grid, cudaStream_t s) {
+  auto kern = decode_split_kernel<FMT, HD, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(p.smem_bytes));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, Fmt<FMT>::kWarps * 32, p.smem_bytes, s>>>(p, tmA, tmB);
+  return cudaGetLastError();
+}
+
+template <int FMT, int HD>
+static cudaError_t launch_g(int G, const DecodeParams& p, const CUtensorMap& tmA,
+                            const CUtensorMap& tmB, int grid, cudaStream_t s) {
+  switch (G) {
+    case 1: return launch_one<FMT, HD, 1>(p, tmA, tmB, grid, s);
+    case 2: return launch_one<FMT, HD, 2>(p, tmA, tmB, grid, s);
+    case 4: return launch_one<FMT, HD, 4>(p, tmA, tmB, grid, s);
+    case 8: return launch_one<FMT, HD, 8>(p, tmA, tmB, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int FMT>
+static cudaError_t launch_hd(int hd, int G, const DecodeParams& p, const CUtensorMap& tmA,
+                             const CUtensorMap& tmB, int grid, cudaStream_t s) {
+  if (hd == 64) return launch_g<FMT, 64>(G, p, tmA, tmB, grid, s);
+  if (hd == 128) return launch_g<FMT, 128>(G, p, tmA, tmB, grid, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
+                          const CUtensorMap& tmA, const CUtensorMap& tmB, int grid,
+                          cudaStream_t s) {
+  switch (fmt) {
+    case STARKV_FMT_F32: return launch_hd<FMT_F32>(head_dim, G, p, tmA, tmB, grid, s);
+    case STARKV_FMT_BF16: return launch_hd<FMT_BF16>(head_dim, G, p, tmA, tmB, grid, s);
+    case STARKV_FMT_MIXED: return launch_hd<FMT_MIXED>(head_dim, G, p, tmA, tmB, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s) {
+  decode_combine_kernel<<<p.batch * p.H, 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+size_t decode_smem_limit() { return 232448; }
+
+}  // namespace starkv

@@ -1,0 +1,94 @@
+// Device-side parameter blocks and launch entry points shared by the kernels and the C ABI.
+#pragma once
+#include "ptx.cuh"
+
+namespace starkv {
+
+constexpr int kTile = STARKV_TILE_TOKENS;  // tokens per decode tile
+constexpr int kPage = 64;                  // tokens per page
+constexpr int kKBytes = 128;               // bytes of K per operand row per k-block
+constexpr int kAStage = kTile * kKBytes;   // 16 KB: one k-block of a 128-row tile
+constexpr int kMaxChunks = 32;             // ceil(64 heads * 128 / 256)
+
+// One latent's description for device code (offsets inside a page; page_bytes < 2^31).
+struct LatDesc {
+  int rank;  // channels
+  int col;   // first column in the concatenated projection
+  int n8, nb4, g8, ng;  // mixed split; ng = g8 + g4
+  int off0;  // plain block (f32/bf16) or int8 block (mixed)
+  int off1;  // packed int4 block (mixed)
+  int off2;  // fp16 scale block (mixed)
+  int pitch; // plain: bytes per token
+};
+
+// Latent store / read-back (quant_pack, append epilogue, dequant).
+struct StoreParams {
+  const float* src;        // [nsplit][n_tok][proj_cols] fp32 (summed in split order)
+  long long split_stride;  // floats between splits
+  int nsplit;
+  float* latents_out;      // optional [n_tok][proj_cols]
+  uint8_t* cache;
+  long long num_pages, page_bytes;
+  const int* block_table;
+  int max_pages, batch;
+  const int* tok_seq;
+  const int* tok_pos;
+  int n_tok;
+  int fmt, n_lat, proj_cols;
+  int* status;
+  LatDesc lat[1 + STARKV_MAX_KV_HEADS];
+};
+
+struct DecodeParams {
+  const uint8_t* cache;
+  long long num_pages, page_bytes;
+  const int* block_table;
+  int max_pages;
+  const int* seq_lens;
+  int batch;
+  const void* q;      // [batch][H][d] bf16 or f32
+  const float* Bv;    // [R_v][d]
+  const float2* rope; // fine [128][d/2] then base [rope_tiles][d/2]
+  int rope_tiles;
+  float* ws;          // partial records
+  int tiles_max, rec; // tiles per sequence slot, floats per record
+  float* out;         // [batch][H][d]
+  int* status;
+  unsigned long long timeout_ns;
+  int H, Hkv, G, d, rk, key_rank_cols;
+  int NC, n_chunks, n_ranges, cpr, kb_count, total_units;
+  uint32_t idesc;
+  float qscale;  // log2(e) / sqrt(d)
+  // dynamic shared-memory plan (offsets from the 1024-aligned base)
+  int stages, nvb, vslot;
+  uint32_t off_b, off_v, off_q, off_p, off_red, off_bar, smem_bytes;
+  LatDesc key;
+  int vchunk_off[kMaxChunks];
+  int vchunk_bytes[kMaxChunks];
+  LatDesc vh[STARKV_MAX_KV_HEADS];
+};
+
+// Launchers (defined in the .cu files; return cudaError_t of the launch).
+cudaError_t launch_store(const StoreParams& p, cudaStream_t s);
+cudaError_t launch_dequant(const StoreParams& p, cudaStream_t s);
+cudaError_t launch_rope_init(float2* table, int half_dim, int rows_fine, int tiles, double theta,
+                             int head_dim, cudaStream_t s);
+cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
+                          const CUtensorMap& tmA, const CUtensorMap& tmB, int grid,
+                          cudaStream_t s);
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s);
+size_t decode_smem_limit();
+
+struct ProjParams {
+  float* part;       // [nsplit][n_tok][proj_cols]
+  int n_tok, proj_cols, d_model;
+  int kb_total, kb_per_split, nsplit;
+  int stages;
+  uint32_t idesc;
+  int* status;
+  unsigned long long timeout_ns;
+};
+cudaError_t launch_project(int fmt, const ProjParams& p, const CUtensorMap& tmX,
+                           const CUtensorMap& tmA, cudaStream_t s);
+
+}  // namespace starkv

@@ -1,0 +1,190 @@
+// Latent storage: fp32 / bf16 / int8+int4 quantisation and packing into cache pages, the
+// read-back (dequantisation) of stored latents, and the RoPE table.
+//
+// Quantiser (per token, per latent, per group of 32 channels; groups restart where the
+// int4 part starts): s16 = fp16_rne(fp32(amax) / qmax) saturated to 65504,
+// code = clamp(rint_half_even(fp32(c) / fp32(s16)), -qmax, qmax), s16 == 0 gives code 0.
+// The leading ceil(r/4) channels (singular-value order: the outlier channels of STAR-KV
+// technical summary, Methodology §3 "Low-Rank-Aware Mixed-Precision Quantization") are int8,
+// the rest int4, two per byte with the even channel in the low nibble.
+#include "internal.cuh"
+
+namespace starkv {
+
+namespace {
+
+__device__ __forceinline__ float warp_max_abs(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// fp16 scale of a group (saturating) and the code of value c.
+__device__ __forceinline__ __half group_scale(float amax, float qmax) {
+  __half h = __float2half_rn(__fdiv_rn(amax, qmax));
+  if (__hisinf(h)) h = __ushort_as_half(static_cast<unsigned short>(0x7BFF));
+  return h;
+}
+__device__ __forceinline__ int quant_code(float c, float s, int qmax) {
+  if (s == 0.f) return 0;
+  const int q = __float2int_rn(__fdiv_rn(c, s));
+  return max(-qmax, min(qmax, q));
+}
+
+struct TokenSlot {
+  uint8_t* page;  // nullptr if the token's page or position is invalid
+  int slot;
+};
+
+__device__ __forceinline__ TokenSlot locate(const StoreParams& p, int n, int li, int lane) {
+  const int b = p.tok_seq[n], pos = p.tok_pos[n];
+  TokenSlot t{nullptr, 0};
+  if (b < 0 || b >= p.batch || pos < 0 || pos >= p.max_pages * kPage) {
+    if (lane == 0 && li == 0 && p.status) atomicOr(p.status, STARKV_DEV_BOUNDS);
+    return t;
+  }
+  const int pg = p.block_table[(long long)b * p.max_pages + pos / kPage];
+  if (pg < 0 || pg >= p.num_pages) {
+    if (lane == 0 && li == 0 && p.status) atomicOr(p.status, STARKV_DEV_BOUNDS);
+    return t;
+  }
+  t.page = p.cache + (long long)pg * p.page_bytes;
+  t.slot = pos % kPage;
+  return t;
+}
+
+// One warp per (token, latent).
+__global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ StoreParams p) {
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= p.n_tok * p.n_lat) return;  // whole warp
+  const int n = gw / p.n_lat, li = gw % p.n_lat;
+  const LatDesc& d = p.lat[li];
+  const TokenSlot ts = locate(p, n, li, lane);
+  const float* src = p.src + (long long)n * p.proj_cols + d.col;
+  auto val = [&](int i) {
+    float v = src[i];
+    for (int s = 1; s < p.nsplit; ++s) v += src[(long long)s * p.split_stride + i];
+    return v;
+  };
+  float* lout = p.latents_out ? p.latents_out + (long long)n * p.proj_cols + d.col : nullptr;
+
+  if (p.fmt == STARKV_FMT_F32 || p.fmt == STARKV_FMT_BF16) {
+    for (int i = lane; i < d.rank; i += 32) {
+      const float c = val(i);
+      if (lout) lout[i] = c;
+      if (!ts.page) continue;
+      uint8_t* dst = ts.page + d.off0 + ts.slot * d.pitch;
+      if (p.fmt == STARKV_FMT_F32)
+        reinterpret_cast<float*>(dst)[i] = c;
+      else
+        reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(c);
+    }
+    return;
+  }
+  __half* sc = ts.page ? reinterpret_cast<__half*>(ts.page + d.off2) + ts.slot * d.ng : nullptr;
+  // int8 part
+  for (int gi = 0; gi < d.g8; ++gi) {
+    const int i = gi * 32 + lane;
+    const bool in = i < d.n8;
+    const float c = in ? val(i) : 0.f;
+    if (lout && in) lout[i] = c;
+    const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
+    const __half h = group_scale(amax, 127.f);
+    const int q = quant_code(c, __half2float(h), 127);
+    if (ts.page && in) reinterpret_cast<int8_t*>(ts.page + d.off0)[ts.slot * d.n8 + i] = static_cast<int8_t>(q);
+    if (ts.page && lane == 0) sc[gi] = h;
+  }
+  // int4 part
+  const int n4 = d.rank - d.n8;
+  for (int gi = 0; gi < d.ng - d.g8; ++gi) {
+    const int j = gi * 32 + lane;
+    const bool in = j < n4;
+    const float c = in ? val(d.n8 + j) : 0.f;
+    if (lout && in) lout[d.n8 + j] = c;
+    const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
+    const __half h = group_scale(amax, 7.f);
+    const int q = quant_code(c, __half2float(h), 7);
+    const int nib = q & 15;
+    const int hi = __shfl_down_sync(0xffffffffu, nib, 1);
+    if (ts.page && in && (j & 1) == 0) {
+      const int byte = nib | ((j + 1 < n4 ? hi : 0) << 4);
+      (ts.page + d.off1)[ts.slot * d.nb4 + (j >> 1)] = static_cast<uint8_t>(byte);
+    }
+    if (ts.page && lane == 0) sc[d.g8 + gi] = h;
+  }
+}
+
+// One warp per (token, latent): stored value -> fp32 (scale * code for the mixed format).
+__global__ void __launch_bounds__(128) dequant_kernel(const __grid_constant__ StoreParams p) {
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= p.n_tok * p.n_lat) return;
+  const int n = gw / p.n_lat, li = gw % p.n_lat;
+  const LatDesc& d = p.lat[li];
+  const TokenSlot ts = locate(p, n, li, lane);
+  float* out = p.latents_out + (long long)n * p.proj_cols + d.col;
+  for (int i = lane; i < d.rank; i += 32) {
+    float v = 0.f;
+    if (ts.page) {
+      const uint8_t* pg = ts.page;
+      if (p.fmt == STARKV_FMT_F32) {
+        v = reinterpret_cast<const float*>(pg + d.off0 + ts.slot * d.pitch)[i];
+      } else if (p.fmt == STARKV_FMT_BF16) {
+        v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(pg + d.off0 + ts.slot * d.pitch)[i]);
+      } else {
+        const __half* sc = reinterpret_cast<const __half*>(pg + d.off2) + ts.slot * d.ng;
+        if (i < d.n8) {
+          const int8_t q = reinterpret_cast<const int8_t*>(pg + d.off0)[ts.slot * d.n8 + i];
+          v = __half2float(sc[i >> 5]) * static_cast<float>(q);
+        } else {
+          const int j = i - d.n8;
+          const uint8_t byte = (pg + d.off1)[ts.slot * d.nb4 + (j >> 1)];
+          const int nib = (j & 1) ? (byte >> 4) : (byte & 15);
+          v = __half2float(sc[d.g8 + (j >> 5)]) * static_cast<float>((nib ^ 8) - 8);
+        }
+      }
+    }
+    out[i] = v;
+  }
+}
+
+// cos/sin of t * theta^(-2j/d) in fp64, stored as fp32: rows 0..127 are t = row (offset
+// inside a 128-token tile), rows 128.. are t = 128 * (row - 128) (tile starts).
+__global__ void rope_init_kernel(float2* table, int half_dim, int rows, double theta,
+                                 int head_dim) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * half_dim) return;
+  const int row = idx / half_dim, j = idx % half_dim;
+  const double t = row < kTile ? static_cast<double>(row) : static_cast<double>(kTile) * (row - kTile);
+  const double inv = pow(theta, -2.0 * static_cast<double>(j) / static_cast<double>(head_dim));
+  double s, c;
+  sincos(t * inv, &s, &c);
+  table[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+}  // namespace
+
+cudaError_t launch_store(const StoreParams& p, cudaStream_t s) {
+  const long long warps = (long long)p.n_tok * p.n_lat;
+  if (warps == 0) return cudaSuccess;
+  store_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const StoreParams& p, cudaStream_t s) {
+  const long long warps = (long long)p.n_tok * p.n_lat;
+  if (warps == 0) return cudaSuccess;
+  dequant_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_init(float2* table, int half_dim, int rows_fine, int tiles, double theta,
+                             int head_dim, cudaStream_t s) {
+  const int rows = rows_fine + tiles;
+  const int total = rows * half_dim;
+  rope_init_kernel<<<(total + 255) / 256, 256, 0, s>>>(table, half_dim, rows, theta, head_dim);
+  return cudaGetLastError();
+}
+
+}  // namespace starkv

@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every entry point the
+header declares, and its pure host calls (layout, sizes, validation) agree with the oracle's
+independent layout definition."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from rank_quantized_kv_decode_b200 import _lib as L
+from rank_quantized_kv_decode_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rank_quantized_kv_decode_b200 import build
+    build.build()
+    return L.load()
+
+
+def declared_entry_points():
+    src = open(os.path.join(ROOT, "include", "starkv.h")).read()
+    return re.findall(r"STARKV_API\s+[\w\s\*]+?\b(starkv_\w+)\s*\(", src)
+
+
+def test_header_declares_the_abi():
+    names = declared_entry_points()
+    assert set(names) == set(L.EXPORTS), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_entry_points():
+        assert hasattr(lib, name), name
+    assert lib.starkv_version() == 100
+
+
+def test_struct_sizes_match_c(lib):
+    # the C side checks that a layout equals starkv_layout_init's output byte for byte,
+    # so a ctypes struct of the wrong size would be rejected
+    assert ctypes.sizeof(L.Config) == 296
+    assert ctypes.sizeof(L.Segment) == 64
+    assert ctypes.sizeof(L.Layout) == 296 + 16 + 16 + 65 * 64
+
+
+CASES = [
+    ("f32", 4, 4, 64, 256, 64, [40, 44, 47, 50]),
+    ("bf16", 32, 32, 128, 4096, 1024, [16 + (g * 7) % 49 for g in range(32)]),
+    ("mixed", 32, 32, 128, 4096, 1024, [16 + (g * 5) % 49 for g in range(32)]),
+    ("mixed", 32, 8, 128, 4096, 256, [8, 48, 37, 17, 32, 29, 40, 45]),
+]
+
+
+@pytest.mark.parametrize("fmt,H,Hkv,d,dm,rk,rv", CASES)
+def test_layout_matches_oracle(lib, fmt, H, Hkv, d, dm, rk, rv):
+    lay = api.layout_init(api.make_config(H, Hkv, d, dm, rk, rv, fmt, 10000.0))
+    ref = O.page_layout(fmt, rk, rv, page_tokens=64)
+    assert lay.page_bytes == ref["page_bytes"]
+    assert lay.token_bytes == ref["token_bytes"]
+    assert lay.n_latents == 1 + Hkv
+    assert lay.proj_cols == rk + sum(rv)
+    col = 0
+    for li, s in enumerate(ref["segs"]):
+        seg = lay.seg[li]
+        assert seg.rank == s["rank"] and seg.col == col
+        col += s["rank"]
+        if fmt == "mixed":
+            assert (seg.n8, seg.n4, seg.g8, seg.g4, seg.nb4) == (s["n8"], s["n4"], s["g8"], s["g4"], s["nb4"])
+            assert (seg.off_i8, seg.off_i4, seg.off_sc) == (s["i8"], s["i4"], s["sc"])
+            assert seg.off_plain == -1
+        else:
+            assert seg.off_plain == s["plain"] and seg.pitch == s["pitch"]
+
+
+def test_alloc_sizes(lib):
+    rv = [8, 48, 37, 17, 32, 29, 40, 45]
+    lay = api.layout_init(api.make_config(32, 8, 128, 4096, 256, rv, "mixed", 500000.0))
+    s = api.alloc(lay, 1000, 4, 16, 8192)
+    assert s.cache_bytes == 1000 * lay.page_bytes
+    # RoPE table: 128 in-tile offsets + one row per 128-token tile, d/2 (cos, sin) pairs each
+    assert s.rope_table_bytes == (128 + 8) * 64 * 8
+    # partial records: 2 + max rank floats, rounded up to 4
+    assert s.decode_workspace_bytes == 4 * 32 * 8 * 52 * 4
+    assert s.append_workspace_bytes >= 8192 * lay.proj_cols * 4
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 96, L.ERR_UNSUPPORTED),
+    ("n_kv_heads", 0, L.ERR_INVALID_ARG),
+    ("n_q_heads", 12, L.ERR_INVALID_ARG),
+    ("key_rank", 100, L.ERR_INVALID_ARG),
+    ("page_tokens", 32, L.ERR_UNSUPPORTED),
+    ("fmt", 7, L.ERR_INVALID_ARG),
+    ("rope_theta", float("nan"), L.ERR_INVALID_ARG),
+])
+def test_layout_rejects(lib, field, value, status):
+    cfg = api.make_config(32, 8, 128, 4096, 256, [32] * 8, "mixed", 500000.0)
+    setattr(cfg, field, value)
+    lay = L.Layout()
+    assert lib.starkv_layout_init(ctypes.byref(cfg), ctypes.byref(lay)) == status
+    assert lib.starkv_last_error()
+
+
+def test_value_rank_out_of_range_rejected(lib):
+    cfg = api.make_config(4, 4, 64, 256, 64, [40, 65, 3, 3], "f32", 10000.0)
+    lay = L.Layout()
+    assert lib.starkv_layout_init(ctypes.byref(cfg), ctypes.byref(lay)) == L.ERR_INVALID_ARG
+
+
+def test_tampered_layout_rejected(lib):
+    lay = api.layout_init(api.make_config(4, 4, 64, 256, 64, [40, 44, 47, 50], "f32", 10000.0))
+    lay.page_bytes += 16
+    s = L.Sizes()
+    assert lib.starkv_alloc(ctypes.byref(lay), 4, 1, 4, 0, ctypes.byref(s)) == L.ERR_INVALID_ARG

@@ -199,3 +199,19 @@ def test_paged_encode_read_roundtrip_with_permuted_table():
                     want = O.store_latents(rows[:, off:off + r], fmt)
                 np.testing.assert_array_equal(Cv[gi], want)
                 off += r
+
+
+def test_vector_quantiser_matches_per_token_definition():
+    g = np.random.default_rng(9)
+    for r in [8, 17, 37, 64, 256]:
+        C = (g.standard_normal((40, r)) * np.exp(-np.arange(r) / 20)).astype(np.float32)
+        C[3] = 0.0
+        C[5, :4] = [1e7, -3e-7, 0, 0]
+        q8, q4, sc = O.quantize_rows(C, r)
+        for n in range(C.shape[0]):
+            a8, a4, asc = O.quantize_latent(C[n], r)
+            assert q8[n].tolist() == a8.tolist()
+            assert q4[n].tolist() == a4.tolist()
+            assert sc[n].view(np.uint16).tolist() == asc.view(np.uint16).tolist()
+        np.testing.assert_array_equal(O.dequantize_rows(q8, q4, sc, r),
+                                      np.stack([O.dequantize_latent(*O.quantize_latent(c, r), r) for c in C]))
