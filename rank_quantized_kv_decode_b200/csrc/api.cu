@@ -373,7 +373,7 @@ starkv_status starkv_append(const starkv_layout* lay, const void* x, int32_t n_t
   pp.n_tok = n_tok;
   pp.proj_cols = lay->proj_cols;
   pp.d_model = lay->cfg.d_model;
-  pp.stages = 4;
+  pp.stages = fmt == STARKV_FMT_F32 ? 2 : 4;  // fp32: hi/lo copies double each stage
   pp.idesc = idesc_make(fmt == STARKV_FMT_F32 ? 2u : 1u, 128, 256);
   pp.status = dev_status;
   pp.timeout_ns = 4000000000ull;
@@ -467,7 +467,8 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   p.rk = c.key_rank;
   p.key_rank_cols = c.key_rank;
   const int ncols = c.n_kv_heads * d;
-  p.NC = ncols >= 256 ? 256 : ncols;
+  // fp32 latents keep hi/lo copies of both operands in shared memory: 128-column chunks
+  p.NC = ncols >= 256 ? (fmt == STARKV_FMT_F32 ? 128 : 256) : ncols;
   p.n_chunks = ceil_div(ncols, p.NC);
   p.kb_count = ceil_div(c.key_rank * es, kKBytes);
   int grid_cap = info.sms;
@@ -521,9 +522,10 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   for (const auto& pl : plans) {
     size_t off = 0;
     const int S = pl[0], NVB = pl[1];
-    off += S * static_cast<size_t>(kAStage);
+    const size_t split = fmt == STARKV_FMT_F32 ? 2 : 1;  // hi/lo copies for 3xTF32
+    off += S * split * static_cast<size_t>(kAStage);
     const size_t off_b = off;
-    off += S * bstage;
+    off += S * split * bstage;
     const size_t off_v = off;
     off += static_cast<size_t>(NVB) * 2 * p.vslot;
     const size_t off_q = off;
@@ -534,7 +536,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     off += 2 * 2 * static_cast<size_t>(QPW) * 4 * 4;
     off = (off + 7) / 8 * 8;
     const size_t off_bar = off;
-    off += (2 * S + 4 + 2 * NVB + 1) * 8 + 16;
+    off += (3 * S + 4 + 2 * NVB + 1) * 8 + 16;
     // alignment slack of the dynamic base; at least 120 KB so that one CTA occupies an SM
     // (each CTA allocates all 512 TMEM columns)
     const size_t total = std::max<size_t>(off + 1024, 120 * 1024);

@@ -81,10 +81,13 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
 template <int FMT>
 struct Fmt {
   static constexpr bool kTmaA = FMT != FMT_MIXED;
+  // fp32 operands: 3xTF32 (hi*hi + hi*lo + lo*hi), the hi/lo split done in shared memory
+  static constexpr bool kSplit = FMT == FMT_F32;
   static constexpr int kKind = FMT == FMT_F32 ? 1 : 0;
   static constexpr int kElem = FMT == FMT_F32 ? 4 : 2;
   static constexpr int kKElems = kKBytes / kElem;  // elements per k-block
-  static constexpr int kWarps = kTmaA ? 12 : 16;
+  static constexpr int kWarps = (kTmaA && !kSplit) ? 12 : 16;
+  static constexpr int kFullCount = kSplit ? 4 : (kTmaA ? 1 : 5);
 };
 
 // Stored value of value-latent channel i of token row ``row`` (0..63) in a staged page slot.
@@ -204,6 +207,9 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages, NVB = p.nvb;
   const uint32_t bstage = static_cast<uint32_t>(p.NC) * kKBytes;
+  // stage strides: the split format keeps hi and lo copies of both operands
+  const uint32_t astride = F::kSplit ? 2 * kAStage : kAStage;
+  const uint32_t bstride = F::kSplit ? 2 * bstage : bstage;
 
   uint8_t* sA = smem;
   uint8_t* sB = smem + p.off_b;
@@ -212,16 +218,17 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   float* sP = reinterpret_cast<float*>(smem + p.off_p);    // [2][QPW][128]
   float* sRed = reinterpret_cast<float*>(smem + p.off_red);  // [2][2][QPW][4]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
-  const int B_FULL = 0, B_EMPTY = S, B_ACCF = 2 * S, B_ACCE = 2 * S + 2, B_VF = 2 * S + 4,
-            B_VE = 2 * S + 4 + NVB, B_TD = 2 * S + 4 + 2 * NVB;
+  const int B_FULL = 0, B_EMPTY = S, B_RAW = 2 * S, B_ACCF = 3 * S, B_ACCE = 3 * S + 2,
+            B_VF = 3 * S + 4, B_VE = 3 * S + 4 + NVB, B_TD = 3 * S + 4 + 2 * NVB;
   // misc: [0] TMEM base, [1] abort flag, [2..3] per-warpgroup stop snapshots
   uint32_t* misc = reinterpret_cast<uint32_t*>(bars + B_TD + 1);
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar(B_FULL + s), F::kTmaA ? 1 : 5);
+      mbar_init(bar(B_FULL + s), F::kFullCount);
       mbar_init(bar(B_EMPTY + s), 1);
+      mbar_init(bar(B_RAW + s), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(B_ACCF + a), 1);
@@ -264,14 +271,15 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             uint32_t bytes = bstage;
             if constexpr (F::kTmaA)
               bytes += (U.page0 >= 0 ? 8192u : 0u) + (U.page1 >= 0 ? 8192u : 0u);
-            const uint32_t fb = bar(B_FULL + stage);
+            // the split format lands raw fp32 tiles that the converters turn into hi/lo
+            const uint32_t fb = bar((F::kSplit ? B_RAW : B_FULL) + stage);
             mbar_arrive_expect_tx(fb, bytes);
             if constexpr (F::kTmaA) {
-              const uint32_t da = smem_u32(sA + stage * kAStage);
+              const uint32_t da = smem_u32(sA + stage * astride);
               if (U.page0 >= 0) tma_load_3d(da, &tmA, fb, kb * F::kKElems, 0, U.page0);
               if (U.page1 >= 0) tma_load_3d(da + 8192, &tmA, fb, kb * F::kKElems, 0, U.page1);
             }
-            tma_load_2d(smem_u32(sB + stage * bstage), &tmB, fb, kb * F::kKElems, c * p.NC);
+            tma_load_2d(smem_u32(sB + stage * bstride), &tmB, fb, kb * F::kKElems, c * p.NC);
             issued |= 1u << stage;
             last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -280,7 +288,8 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       }
       // every copy this thread started has landed before the CTA may exit
       for (int s = 0; s < S; ++s)
-        if (issued & (1u << s)) wait_drain(bar(B_FULL + s), (last_phase >> s) & 1u, p.timeout_ns);
+        if (issued & (1u << s))
+          wait_drain(bar((F::kSplit ? B_RAW : B_FULL) + s), (last_phase >> s) & 1u, p.timeout_ns);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -298,11 +307,18 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           for (int kb = 0; kb < p.kb_count; ++kb) {
             if (!wait_bounded(bar(B_FULL + stage), phase, wc)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t da = desc_sw128(smem_u32(sA + stage * kAStage));
-            const uint64_t db = desc_sw128(smem_u32(sB + stage * bstage));
+            const uint64_t da = desc_sw128(smem_u32(sA + stage * astride));
+            const uint64_t db = desc_sw128(smem_u32(sB + stage * bstride));
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 4; ++k) {
               umma<F::kKind>(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
+              if constexpr (F::kSplit) {
+                const uint64_t dal = desc_sw128(smem_u32(sA + stage * astride + kAStage));
+                const uint64_t dbl = desc_sw128(smem_u32(sB + stage * bstride + bstage));
+                umma<F::kKind>(d_tmem, da + 2 * k, dbl + 2 * k, p.idesc, 1u);
+                umma<F::kKind>(d_tmem, dal + 2 * k, db + 2 * k, p.idesc, 1u);
+              }
+            }
             umma_commit(bar(B_EMPTY + stage));
             if (++stage == S) { stage = 0; phase ^= 1u; }
           }
@@ -360,6 +376,8 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     // Control flow of a warpgroup only changes on a snapshot every thread reads after a
     // named barrier, so no thread can leave while the others wait at a barrier.
     bool stop = false;
+    // head slots of this warpgroup that belong to a chunk (NC may be 128: then only WG 0)
+    const int wg_slots = max(0, min(HPW, p.NC / HD - wg * HPW));
     for (int u = blockIdx.x; !stop && u < p.total_units; u += gridDim.x) {
       Unit U;
       if (!get_unit(p, u, U, false)) continue;
@@ -373,7 +391,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         for (int idx = row; idx < QPW * HALF; idx += 128) {
           const int hq = idx / HALF, j = idx % HALF;
           const int g = g_first + hq / G;
-          if (g >= p.Hkv) continue;
+          if (g >= p.Hkv || hq / G >= wg_slots) continue;
           const int h = g * G + hq % G;
           const long long qb = ((long long)U.b * p.H + h) * HD;
           const float x0 = qload<FMT>(p.q, qb + j), x1 = qload<FMT>(p.q, qb + j + HALF);
@@ -394,7 +412,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           float acc[G];
 #pragma unroll
           for (int gq = 0; gq < G; ++gq) acc[gq] = 0.f;
-          if (g_first + hs < p.Hkv) {
+          if (g_first + hs < p.Hkv && hs < wg_slots) {
             const uint32_t taddr = tmem + static_cast<uint32_t>(ab * 256 + wg * 128 + hs * HD) +
                                    (static_cast<uint32_t>(quad * 32) << 16);
 #pragma unroll 1
@@ -450,7 +468,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           const int g = g_first + hs;
-          if (g >= p.Hkv) continue;
+          if (g >= p.Hkv || hs >= wg_slots) continue;
           const LatDesc& vd = p.vh[g];
           if (row < vd.rank) {
             float a[G];
@@ -493,6 +511,35 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       }
     }
   } else if (warp >= 12) {
+    if constexpr (F::kSplit) {
+      // ---------------------------------------------------------------- tf32 hi/lo splitters
+      const int tid = (warp - 12) * 32 + lane;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+        Unit U;
+        if (!get_unit(p, u, U, false)) continue;
+        for (int c = U.c0; ok && c < U.c1; ++c) {
+          for (int kb = 0; kb < p.kb_count; ++kb) {
+            if (!__all_sync(0xffffffffu, wait_bounded(bar(B_RAW + stage), phase, wc))) {
+              ok = false;
+              break;
+            }
+            uint8_t* a = sA + stage * astride;
+            uint8_t* b = sB + stage * bstride;
+            split_tf32(reinterpret_cast<float4*>(a), reinterpret_cast<float4*>(a + kAStage),
+                       kAStage / 16, tid, 128);
+            split_tf32(reinterpret_cast<float4*>(b), reinterpret_cast<float4*>(b + bstage),
+                       static_cast<int>(bstage / 16), tid, 128);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_FULL + stage));
+            if (++stage == S) { stage = 0; phase ^= 1u; }
+          }
+        }
+      }
+    }
     // ---------------------------------------------------------------- dequantisers (int8/int4)
     if constexpr (!F::kTmaA) {
       const int tid = (warp - 12) * 32 + lane;

@@ -12,22 +12,33 @@ namespace starkv {
 namespace {
 
 template <int FMT>
-__global__ void __launch_bounds__(192, 1)
+struct ProjFmt {
+  // fp32 operands run as 3xTF32: hi/lo copies of both tiles, split in shared memory by
+  // four extra warps
+  static constexpr bool kSplit = FMT == STARKV_FMT_F32;
+  static constexpr int kThreads = kSplit ? 320 : 192;
+};
+
+template <int FMT>
+__global__ void __launch_bounds__(ProjFmt<FMT>::kThreads, 1)
     project_kernel(const __grid_constant__ ProjParams p, const __grid_constant__ CUtensorMap tmX,
                    const __grid_constant__ CUtensorMap tmA) {
+  constexpr bool kSplit = ProjFmt<FMT>::kSplit;
   constexpr int kKind = FMT == STARKV_FMT_F32 ? 1 : 0;
   constexpr int kKElems = FMT == STARKV_FMT_F32 ? 32 : 64;
   constexpr uint32_t kBStage = 256 * kKBytes;
+  constexpr uint32_t kAStride = kSplit ? 2 * kAStage : kAStage;
+  constexpr uint32_t kBStride = kSplit ? 2 * kBStage : kBStage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int S = p.stages;
   uint8_t* sA = smem;
-  uint8_t* sB = smem + S * kAStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * kBStage);
-  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 2 * S + 2);
+  uint8_t* sB = smem + S * kAStride;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * kBStride);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 3 * S + 2);
   auto bar = [&](int i) { return smem_u32(bars + i); };
-  const int B_FULL = 0, B_EMPTY = S, B_ACC = 2 * S, B_TD = 2 * S + 1;
+  const int B_FULL = 0, B_EMPTY = S, B_RAW = 2 * S, B_ACC = 3 * S, B_TD = 3 * S + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128, n0 = blockIdx.y * 256;
   const int kb0 = blockIdx.z * p.kb_per_split;
@@ -35,8 +46,9 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_FULL + s), kSplit ? 4 : 1);
       mbar_init(bar(B_EMPTY + s), 1);
+      mbar_init(bar(B_RAW + s), 1);
     }
     mbar_init(bar(B_ACC), 1);
     mbar_init(bar(B_TD), 1);
@@ -61,10 +73,10 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0, issued = 0, last_phase = 0;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_bounded(bar(B_EMPTY + stage), phase ^ 1u, wc)) break;
-        const uint32_t fb = bar(B_FULL + stage);
+        const uint32_t fb = bar((kSplit ? B_RAW : B_FULL) + stage);
         mbar_arrive_expect_tx(fb, kAStage + kBStage);
-        tma_load_2d(smem_u32(sA + stage * kAStage), &tmX, fb, kb * kKElems, m0);
-        tma_load_2d(smem_u32(sB + stage * kBStage), &tmA, fb, kb * kKElems, n0);
+        tma_load_2d(smem_u32(sA + stage * kAStride), &tmX, fb, kb * kKElems, m0);
+        tma_load_2d(smem_u32(sB + stage * kBStride), &tmA, fb, kb * kKElems, n0);
         issued |= 1u << stage;
         last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -72,7 +84,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int s = 0; s < S; ++s) {
         if (!(issued & (1u << s))) continue;
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(bar(B_FULL + s), (last_phase >> s) & 1u))
+        while (!mbar_try_wait(bar((kSplit ? B_RAW : B_FULL) + s), (last_phase >> s) & 1u))
           if (globaltimer_ns() - t0 > p.timeout_ns) break;
       }
     }
@@ -85,10 +97,18 @@ __global__ void __launch_bounds__(192, 1)
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_bounded(bar(B_FULL + stage), phase, wc)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t da = desc_sw128(smem_u32(sA + stage * kAStage));
-        const uint64_t db = desc_sw128(smem_u32(sB + stage * kBStage));
+        const uint64_t da = desc_sw128(smem_u32(sA + stage * kAStride));
+        const uint64_t db = desc_sw128(smem_u32(sB + stage * kBStride));
 #pragma unroll
-        for (int k = 0; k < 4; ++k) umma<kKind>(tmem, da + 2 * k, db + 2 * k, idesc, (kb > kb0 || k > 0));
+        for (int k = 0; k < 4; ++k) {
+          umma<kKind>(tmem, da + 2 * k, db + 2 * k, idesc, (kb > kb0 || k > 0));
+          if constexpr (kSplit) {
+            const uint64_t dal = desc_sw128(smem_u32(sA + stage * kAStride + kAStage));
+            const uint64_t dbl = desc_sw128(smem_u32(sB + stage * kBStride + kBStage));
+            umma<kKind>(tmem, da + 2 * k, dbl + 2 * k, idesc, 1u);
+            umma<kKind>(tmem, dal + 2 * k, db + 2 * k, idesc, 1u);
+          }
+        }
         umma_commit(bar(B_EMPTY + stage));
         if (++stage == S) { stage = 0; phase ^= 1u; }
       }
@@ -99,6 +119,26 @@ __global__ void __launch_bounds__(192, 1)
         if (globaltimer_ns() - t0 > p.timeout_ns) break;
     }
     __syncwarp();
+  } else if (warp >= 6) {
+    if constexpr (kSplit) {
+      // tf32 hi/lo splitters (warps 6..9)
+      const int tid = (warp - 6) * 32 + lane;
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!__all_sync(0xffffffffu, wait_bounded(bar(B_RAW + stage), phase, wc))) break;
+        uint8_t* a = sA + stage * kAStride;
+        uint8_t* b = sB + stage * kBStride;
+        split_tf32(reinterpret_cast<float4*>(a), reinterpret_cast<float4*>(a + kAStage),
+                   kAStage / 16, tid, 128);
+        split_tf32(reinterpret_cast<float4*>(b), reinterpret_cast<float4*>(b + kBStage),
+                   kBStage / 16, tid, 128);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_FULL + stage));
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+    }
   } else {
     // epilogue: warps 2..5 cover TMEM lane quadrants 2, 3, 0, 1
     const int quad = warp & 3;
@@ -140,14 +180,15 @@ cudaError_t launch_project(int fmt, const ProjParams& p, const CUtensorMap& tmX,
   const int m_tiles = (p.n_tok + 127) / 128;
   const int n_tiles = (p.proj_cols + 255) / 256;
   dim3 grid(m_tiles, n_tiles, p.nsplit);
-  const size_t smem = 1024 + static_cast<size_t>(p.stages) * (kAStage + 256 * kKBytes) +
-                      (2 * p.stages + 2) * 8 + 16;
+  const size_t split = fmt == STARKV_FMT_F32 ? 2 : 1;
+  const size_t smem = 1024 + static_cast<size_t>(p.stages) * split * (kAStage + 256 * kKBytes) +
+                      (3 * p.stages + 2) * 8 + 16;
   cudaError_t e;
   if (fmt == STARKV_FMT_F32) {
     e = cudaFuncSetAttribute(project_kernel<STARKV_FMT_F32>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    project_kernel<STARKV_FMT_F32><<<grid, 192, smem, s>>>(p, tmX, tmA);
+    project_kernel<STARKV_FMT_F32><<<grid, ProjFmt<STARKV_FMT_F32>::kThreads, smem, s>>>(p, tmX, tmA);
   } else {
     e = cudaFuncSetAttribute(project_kernel<STARKV_FMT_BF16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

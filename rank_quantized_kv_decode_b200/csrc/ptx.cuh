@@ -192,6 +192,26 @@ __device__ __forceinline__ void tmem_ld32x2_wait(uint32_t taddr0, uint32_t taddr
   }
 }
 
+// Nearest tf32 value (ties away from zero) of an fp32 value, returned as fp32 with the low 13
+// mantissa bits clear.  x - tf32_round(x) is exact in fp32 and is the "lo" part of a 3xTF32
+// product split: a*b ~= a_hi*b_hi + a_hi*b_lo + a_lo*b_hi (relative error ~2^-21).
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// Split ``n16`` 16-byte chunks of fp32 values in place into hi (kept at ``buf``) and lo
+// (written at ``lo``), thread ``t`` of ``nthreads``.  Layout-agnostic: works on any swizzle.
+__device__ __forceinline__ void split_tf32(float4* buf, float4* lo, int n16, int t, int nthreads) {
+  for (int i = t; i < n16; i += nthreads) {
+    float4 v = buf[i];
+    float4 h = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z), tf32_round(v.w));
+    buf[i] = h;
+    lo[i] = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+  }
+}
+
 // Shared-memory matrix descriptor of a K-major operand tile stored with the 128-byte
 // swizzle: rows of 128 bytes, 8-row atoms of 1024 bytes (stride-byte-offset 1024), tile
 // base 1024-byte aligned.  Advancing K by 32 bytes inside the atom adds 2 to the result.
