@@ -534,7 +534,9 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     off += 2 * static_cast<size_t>(QPW) * kTile * 4;
     const size_t off_red = off;
     off += 2 * 2 * static_cast<size_t>(QPW) * 4 * 4;
-    off = (off + 7) / 8 * 8;
+    off = (off + 15) / 16 * 16;
+    const size_t off_ang = off;
+    off += 2 * 2 * static_cast<size_t>(d / 2) * 4;
     const size_t off_bar = off;
     off += (3 * S + 4 + 2 * NVB + 1) * 8 + 16;
     // alignment slack of the dynamic base; at least 120 KB so that one CTA occupies an SM
@@ -548,6 +550,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
       p.off_q = static_cast<uint32_t>(off_q);
       p.off_p = static_cast<uint32_t>(off_p);
       p.off_red = static_cast<uint32_t>(off_red);
+      p.off_ang = static_cast<uint32_t>(off_ang);
       p.off_bar = static_cast<uint32_t>(off_bar);
       p.smem_bytes = static_cast<uint32_t>(total);
       planned = true;

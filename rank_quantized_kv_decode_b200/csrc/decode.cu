@@ -217,6 +217,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   float* sQ = reinterpret_cast<float*>(smem + p.off_q);    // [2][QPW][HD]
   float* sP = reinterpret_cast<float*>(smem + p.off_p);    // [2][QPW][128]
   float* sRed = reinterpret_cast<float*>(smem + p.off_red);  // [2][2][QPW][4]
+  float* sAng = reinterpret_cast<float*>(smem + p.off_ang);  // [2][2][HALF]: theta_j, tile angle
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   const int B_FULL = 0, B_EMPTY = S, B_RAW = 2 * S, B_ACCF = 3 * S, B_ACCE = 3 * S + 2,
             B_VF = 3 * S + 4, B_VE = 3 * S + 4 + NVB, B_TD = 3 * S + 4 + 2 * NVB;
@@ -367,6 +368,16 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     const int row = quad * 32 + lane;   // token row in the tile == thread index in the WG
     const float2* fine = p.rope;
     const float2* basetab = p.rope + kTile * HALF;
+    // RoPE angles of this warpgroup: theta_j (fixed) and the tile-start angle phi_j, both
+    // recovered from the fp64-built table; a row's angle phi_j + r*theta_j stays below
+    // pi + 128, where the SFU sine/cosine error is ~1e-5 rad -- no per-element table reads
+    float* theta_s = sAng + wg * 2 * HALF;
+    float* phi_s = theta_s + HALF;
+    for (int j = row; j < HALF; j += 128) {
+      const float2 f1 = fine[HALF + j];  // row 1: angle theta_j
+      theta_s[j] = atan2f(f1.y, f1.x);
+    }
+    const float rowf = static_cast<float>(row);
     float* q_s = sQ + wg * QPW * HD;
     float* p_s = sP + wg * QPW * kTile;
     float* red = sRed + wg * 2 * QPW * 4;
@@ -383,11 +394,13 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       if (!get_unit(p, u, U, false)) continue;
       const int T = U.L - 1;  // position of the decode query
       const bool rv = row < U.nvalid && U.page(row >> 6) >= 0;
-      const float2* fine_r = fine + row * HALF;
-      const float2* base_t = basetab + U.tile * HALF;
       for (int c = U.c0; c < U.c1; ++c) {
         const int g_first = c * (p.NC / HD) + wg * HPW;
-        // (1) rotated, scaled queries of this warpgroup's heads
+        // (1) rotated, scaled queries of this warpgroup's heads; the tile's start angles
+        for (int j = row; j < HALF; j += 128) {
+          const float2 bs = basetab[U.tile * HALF + j];
+          phi_s[j] = atan2f(bs.y, bs.x);
+        }
         for (int idx = row; idx < QPW * HALF; idx += 128) {
           const int hq = idx / HALF, j = idx % HALF;
           const int g = g_first + hq / G;
@@ -416,19 +429,37 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             const uint32_t taddr = tmem + static_cast<uint32_t>(ab * 256 + wg * 128 + hs * HD) +
                                    (static_cast<uint32_t>(quad * 32) << 16);
 #pragma unroll 1
-            for (int jj = 0; jj < HALF; jj += 32) {
-              float klo[32], khi[32];
-              tmem_ld32x2_wait(taddr + jj, taddr + HALF + jj, klo, khi);
+            for (int jj = 0; jj < HALF; jj += 16) {
+              float klo[16], khi[16];
+              tmem_ld16x2_wait(taddr + jj, taddr + HALF + jj, klo, khi);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float2 f = fine_r[jj + j], bs = base_t[jj + j];
-                const float cs = bs.x * f.x - bs.y * f.y, sn = bs.y * f.x + bs.x * f.y;
-                const float k0 = klo[j] * cs - khi[j] * sn;
-                const float k1 = khi[j] * cs + klo[j] * sn;
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const int j0 = jj + 4 * j4;
+                const float4 th = *reinterpret_cast<const float4*>(theta_s + j0);
+                const float4 ph = *reinterpret_cast<const float4*>(phi_s + j0);
+                float cs[4], sn[4];
+                __sincosf(fmaf(rowf, th.x, ph.x), &sn[0], &cs[0]);
+                __sincosf(fmaf(rowf, th.y, ph.y), &sn[1], &cs[1]);
+                __sincosf(fmaf(rowf, th.z, ph.z), &sn[2], &cs[2]);
+                __sincosf(fmaf(rowf, th.w, ph.w), &sn[3], &cs[3]);
+                float k0[4], k1[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float a = klo[4 * j4 + e], b = khi[4 * j4 + e];
+                  k0[e] = a * cs[e] - b * sn[e];
+                  k1[e] = b * cs[e] + a * sn[e];
+                }
 #pragma unroll
                 for (int gq = 0; gq < G; ++gq) {
-                  const float* qq = q_s + (hs * G + gq) * HD + jj + j;
-                  acc[gq] = fmaf(k0, qq[0], fmaf(k1, qq[HALF], acc[gq]));
+                  const float* qq = q_s + (hs * G + gq) * HD + j0;
+                  const float4 qa = *reinterpret_cast<const float4*>(qq);
+                  const float4 qb = *reinterpret_cast<const float4*>(qq + HALF);
+                  float t = acc[gq];
+                  t = fmaf(k0[0], qa.x, t); t = fmaf(k1[0], qb.x, t);
+                  t = fmaf(k0[1], qa.y, t); t = fmaf(k1[1], qb.y, t);
+                  t = fmaf(k0[2], qa.z, t); t = fmaf(k1[2], qb.z, t);
+                  t = fmaf(k0[3], qa.w, t); t = fmaf(k1[3], qb.w, t);
+                  acc[gq] = t;
                 }
               }
             }
