@@ -154,7 +154,15 @@ void fill_store(StoreParams& sp, const starkv_layout* lay) {
   sp.fmt = lay->cfg.fmt;
   sp.n_lat = lay->n_latents;
   sp.proj_cols = lay->proj_cols;
-  for (int i = 0; i < lay->n_latents; ++i) sp.lat[i] = lat_desc(lay->seg[i]);
+  int chunks = 0;
+  for (int i = 0; i < lay->n_latents; ++i) {
+    sp.lat[i] = lat_desc(lay->seg[i]);
+    sp.chunk_start[i] = static_cast<short>(chunks);
+    const starkv_segment& g = lay->seg[i];
+    chunks += lay->cfg.fmt == STARKV_FMT_MIXED ? g.g8 + g.g4 : (g.rank + 31) / 32;
+  }
+  sp.chunk_start[lay->n_latents] = static_cast<short>(chunks);
+  sp.chunks_per_token = chunks;
 }
 
 }  // namespace

@@ -36,7 +36,9 @@ struct StoreParams {
   int n_tok;
   int fmt, n_lat, proj_cols;
   int* status;
+  int chunks_per_token;  // sum over latents of their 32-channel chunks (one warp each)
   LatDesc lat[1 + STARKV_MAX_KV_HEADS];
+  short chunk_start[2 + STARKV_MAX_KV_HEADS];  // first chunk index of each latent
 };
 
 struct DecodeParams {

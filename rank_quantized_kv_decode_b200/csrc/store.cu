@@ -53,54 +53,71 @@ __device__ __forceinline__ TokenSlot locate(const StoreParams& p, int n, int li,
   return t;
 }
 
-// One warp per (token, latent).
+// Sum of the split-K partials of one value, in split order (deterministic).  The loads are
+// issued before the adds so they are in flight together.
+__device__ __forceinline__ float split_sum(const float* src, long long stride, int nsplit) {
+  float v = src[0];
+  int s = 1;
+  for (; s + 4 <= nsplit; s += 4) {
+    const float a = src[s * stride], b = src[(s + 1) * stride];
+    const float c = src[(s + 2) * stride], d = src[(s + 3) * stride];
+    v += a;
+    v += b;
+    v += c;
+    v += d;
+  }
+  for (; s < nsplit; ++s) v += src[s * stride];
+  return v;
+}
+
+// One warp per (token, latent, 32-channel chunk): lane = channel.  In the int8/int4 format a
+// chunk is one quantisation group (the int8 groups, then the int4 groups of the latent).
 __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ StoreParams p) {
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (gw >= p.n_tok * p.n_lat) return;  // whole warp
-  const int n = gw / p.n_lat, li = gw % p.n_lat;
+  if (gw >= p.n_tok * p.chunks_per_token) return;  // whole warp
+  const int n = gw / p.chunks_per_token;
+  const int ck = gw % p.chunks_per_token;
+  int li = 0;
+  while (p.chunk_start[li + 1] <= ck) ++li;
+  const int cl = ck - p.chunk_start[li];  // chunk within the latent
   const LatDesc& d = p.lat[li];
-  const TokenSlot ts = locate(p, n, li, lane);
+  const TokenSlot ts = locate(p, n, (li == 0 && cl == 0) ? 0 : 1, lane);
   const float* src = p.src + (long long)n * p.proj_cols + d.col;
-  auto val = [&](int i) {
-    float v = src[i];
-    for (int s = 1; s < p.nsplit; ++s) v += src[(long long)s * p.split_stride + i];
-    return v;
-  };
   float* lout = p.latents_out ? p.latents_out + (long long)n * p.proj_cols + d.col : nullptr;
 
   if (p.fmt == STARKV_FMT_F32 || p.fmt == STARKV_FMT_BF16) {
-    for (int i = lane; i < d.rank; i += 32) {
-      const float c = val(i);
-      if (lout) lout[i] = c;
-      if (!ts.page) continue;
-      uint8_t* dst = ts.page + d.off0 + ts.slot * d.pitch;
-      if (p.fmt == STARKV_FMT_F32)
-        reinterpret_cast<float*>(dst)[i] = c;
-      else
-        reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(c);
-    }
+    const int i = cl * 32 + lane;
+    if (i >= d.rank) return;
+    const float c = split_sum(src + i, p.split_stride, p.nsplit);
+    if (lout) lout[i] = c;
+    if (!ts.page) return;
+    uint8_t* dst = ts.page + d.off0 + ts.slot * d.pitch;
+    if (p.fmt == STARKV_FMT_F32)
+      reinterpret_cast<float*>(dst)[i] = c;
+    else
+      reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(c);
     return;
   }
   __half* sc = ts.page ? reinterpret_cast<__half*>(ts.page + d.off2) + ts.slot * d.ng : nullptr;
-  // int8 part
-  for (int gi = 0; gi < d.g8; ++gi) {
-    const int i = gi * 32 + lane;
+  if (cl < d.g8) {
+    // int8 group cl: channels [32 cl, min(32 cl + 32, n8))
+    const int i = cl * 32 + lane;
     const bool in = i < d.n8;
-    const float c = in ? val(i) : 0.f;
+    const float c = in ? split_sum(src + i, p.split_stride, p.nsplit) : 0.f;
     if (lout && in) lout[i] = c;
     const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
     const __half h = group_scale(amax, 127.f);
     const int q = quant_code(c, __half2float(h), 127);
     if (ts.page && in) reinterpret_cast<int8_t*>(ts.page + d.off0)[ts.slot * d.n8 + i] = static_cast<int8_t>(q);
-    if (ts.page && lane == 0) sc[gi] = h;
-  }
-  // int4 part
-  const int n4 = d.rank - d.n8;
-  for (int gi = 0; gi < d.ng - d.g8; ++gi) {
+    if (ts.page && lane == 0) sc[cl] = h;
+  } else {
+    // int4 group gi: channels n8 + [32 gi, min(32 gi + 32, n4))
+    const int gi = cl - d.g8;
+    const int n4 = d.rank - d.n8;
     const int j = gi * 32 + lane;
     const bool in = j < n4;
-    const float c = in ? val(d.n8 + j) : 0.f;
+    const float c = in ? split_sum(src + d.n8 + j, p.split_stride, p.nsplit) : 0.f;
     if (lout && in) lout[d.n8 + j] = c;
     const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
     const __half h = group_scale(amax, 7.f);
@@ -166,7 +183,7 @@ __global__ void rope_init_kernel(float2* table, int half_dim, int rows, double t
 }  // namespace
 
 cudaError_t launch_store(const StoreParams& p, cudaStream_t s) {
-  const long long warps = (long long)p.n_tok * p.n_lat;
+  const long long warps = (long long)p.n_tok * p.chunks_per_token;
   if (warps == 0) return cudaSuccess;
   store_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, s>>>(p);
   return cudaGetLastError();
