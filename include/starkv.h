@@ -231,6 +231,28 @@ STARKV_API starkv_status starkv_decode_combine(const starkv_layout* lay, const i
                                                const void* workspace, size_t workspace_bytes,
                                                float* out, starkv_stream_t stream);
 
+/* starkv_decode_attention without a workspace argument, for callers that cannot allocate
+ * device memory: a plugin inside a host process whose memory pool has already reserved the
+ * GPU's memory, a C caller with no device allocator, or a loop where a cudaMalloc is not
+ * acceptable because it may synchronise the device.  (The pages describe no such interface;
+ * it has no counterpart there.)
+ *   - The partial records live in a 16 MiB array inside the library's device image; every
+ *     GPU that loads the library holds it until the process exits.  Calls whose records need
+ *     more (batch * n_q_heads * ceil(max_pages / 2) * 4 * ceil((2 + value_rank_max) / 4)
+ *     floats) return STARKV_ERR_WORKSPACE with a message; nothing is launched.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents.  Nothing in it needs
+ *     to start at zero: each call writes every record it reads.  Calls whose kernels overlap
+ *     on the GPU (two streams, two threads, two graphs) race on it.
+ *   - Allocates nothing (no cudaMalloc / cudaFree).  Other arguments, results and errors as
+ *     starkv_decode_attention. */
+STARKV_API starkv_status starkv_decode_attention_noalloc(
+    const starkv_layout* lay, const void* q, const void* cache, int64_t num_pages,
+    const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t batch,
+    const void* Bk_t, const float* Bv, const void* rope_table, size_t rope_table_bytes, float* out,
+    const starkv_decode_opts* opts, int32_t* dev_status, starkv_stream_t stream);
+
 /* One-line description of the last non-OK return on this thread. */
 STARKV_API const char* starkv_last_error(void);
 

@@ -64,6 +64,9 @@ EXPORTS = {
     "starkv_decode_partials": (i32, [ctypes.POINTER(Layout), vp, vp, i64, vp, i32, vp, i32, vp, vp,
                                      sz, vp, sz, ctypes.POINTER(DecodeOpts), vp, vp]),
     "starkv_decode_combine": (i32, [ctypes.POINTER(Layout), vp, i32, i32, vp, vp, sz, vp, vp]),
+    "starkv_decode_attention_noalloc": (i32, [ctypes.POINTER(Layout), vp, vp, i64, vp, i32, vp, i32,
+                                              vp, vp, vp, sz, vp, ctypes.POINTER(DecodeOpts), vp,
+                                              vp]),
     "starkv_last_error": (ctypes.c_char_p, []),
     "starkv_version": (i32, []),
 }

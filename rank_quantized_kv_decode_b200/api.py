@@ -103,6 +103,20 @@ def decode_attention(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rope_table,
         _ptr(status), _stream(stream)), "starkv_decode_attention")
 
 
+def decode_attention_noalloc(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rope_table, out,
+                             status, max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
+                             stream=None) -> None:
+    """decode_attention with the library's built-in 16 MiB scratch instead of a workspace
+    (for callers that cannot allocate device memory; see include/starkv.h)."""
+    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms)
+    L.check(L.load().starkv_decode_attention_noalloc(
+        ctypes.byref(lay), _ptr(q), _ptr(cache),
+        cache.numel() * cache.element_size() // lay.page_bytes, _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], _ptr(Bk_t), _ptr(Bv),
+        _ptr(rope_table), rope_table.numel() * rope_table.element_size(), _ptr(out),
+        ctypes.byref(opts), _ptr(status), _stream(stream)), "starkv_decode_attention_noalloc")
+
+
 def decode_partials(lay, q, cache, block_table, seq_lens, Bk_t, rope_table, workspace, status,
                     max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
                     stream=None) -> None:

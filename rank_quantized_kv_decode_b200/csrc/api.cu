@@ -167,6 +167,10 @@ void fill_store(StoreParams& sp, const starkv_layout* lay) {
 
 }  // namespace
 
+namespace starkv {
+void set_error_message(const std::string& msg) { g_last_error = msg; }
+}  // namespace starkv
+
 extern "C" {
 
 const char* starkv_last_error(void) { return g_last_error.c_str(); }

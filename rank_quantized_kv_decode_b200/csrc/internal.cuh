@@ -1,5 +1,7 @@
 // Device-side parameter blocks and launch entry points shared by the kernels and the C ABI.
 #pragma once
+#include <string>
+
 #include "ptx.cuh"
 
 namespace starkv {
@@ -69,6 +71,9 @@ struct DecodeParams {
   int vchunk_bytes[kMaxChunks];
   LatDesc vh[STARKV_MAX_KV_HEADS];
 };
+
+// Sets the message starkv_last_error() returns on this thread (defined with the C ABI).
+void set_error_message(const std::string& msg);
 
 // Launchers (defined in the .cu files; return cudaError_t of the launch).
 cudaError_t launch_store(const StoreParams& p, cudaStream_t s);
