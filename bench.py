@@ -204,6 +204,7 @@ def main():
     from datetime import timedelta
 
     from rank_quantized_kv_decode_b200 import api
+    from rank_quantized_kv_decode_b200 import dist as D
     from rank_quantized_kv_decode_b200 import workload as W
 
     torch.cuda.set_device(local)
@@ -275,14 +276,11 @@ def main():
     split_ms = [e[1].elapsed_time(e[2]) for e in evs]
     if world > 1:
         dist.barrier()
-    total_ms = float(np.sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    # device time of the K steps, max over ranks; every rank processed B sequences
+    total_ms = D.max_over_ranks(float(np.sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
     tokens_per_step = B * L * world
-    value = tokens_per_step / (ms_per_step / 1000.0)
+    value = D.aggregate_rate(B * L * args.steps, world, total_ms / 1000.0)
 
     # end to end through the public API: host inputs (pinned) in, output back to the host
     x_host = x_new.cpu().pin_memory()
@@ -309,12 +307,8 @@ def main():
         e2e_step()
         e2e_evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_total = float(np.sum([a.elapsed_time(b) for a, b in e2e_evs]))
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = tokens_per_step / (e2e_total / args.steps / 1000.0)
+    e2e_total = D.max_over_ranks(float(np.sum([a.elapsed_time(b) for a, b in e2e_evs])), dev)
+    e2e_value = D.aggregate_rate(B * L * args.steps, world, e2e_total / 1000.0)
     h2d = x_host.numel() * x_host.element_size() + q_host.numel() * q_host.element_size()
     d2h = out_host.numel() * out_host.element_size()
     assert lc.status.item() == 0
