@@ -130,6 +130,9 @@ typedef struct {
   int32_t n_ranges;   /* split of the KV heads of one 128-token tile into this many work
                          units; 0 = chosen from the grid size                             */
   int32_t timeout_ms; /* bound of every in-kernel wait; 0 = 4000 ms                       */
+  int32_t cta_group;  /* 0 = auto; 1 = one CTA per 128-token tile; 2 = a pair of CTAs (one
+                         cluster) per 256-token tile sharing each B_k k-block (bf16 and
+                         int8/int4 latents, 256-column chunks)                             */
 } starkv_decode_opts;
 
 /* Fill ``out`` from ``cfg``: per-latent mixed split, block offsets, page size.
@@ -252,6 +255,13 @@ STARKV_API starkv_status starkv_decode_attention_noalloc(
     const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t batch,
     const void* Bk_t, const float* Bv, const void* rope_table, size_t rope_table_bytes, float* out,
     const starkv_decode_opts* opts, int32_t* dev_status, starkv_stream_t stream);
+
+/* Failure-detection check of the in-kernel bounded waits: one CTA holds TMEM and waits on a
+ * barrier that nothing completes.  After ``timeout_ms`` (1..10000) the wait gives up, the CTA
+ * sets STARKV_DEV_TIMEOUT in *dev_status, releases TMEM and returns; the context stays usable.
+ * Device code of every kernel here waits through the same helper. */
+STARKV_API starkv_status starkv_diag_bounded_wait(int32_t timeout_ms, int32_t* dev_status,
+                                                  starkv_stream_t stream);
 
 /* One-line description of the last non-OK return on this thread. */
 STARKV_API const char* starkv_last_error(void);

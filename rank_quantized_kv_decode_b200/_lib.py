@@ -45,7 +45,7 @@ class Sizes(ctypes.Structure):
 
 
 class DecodeOpts(ctypes.Structure):
-    _fields_ = [("max_ctas", i32), ("n_ranges", i32), ("timeout_ms", i32)]
+    _fields_ = [("max_ctas", i32), ("n_ranges", i32), ("timeout_ms", i32), ("cta_group", i32)]
 
 
 EXPORTS = {
@@ -67,6 +67,7 @@ EXPORTS = {
     "starkv_decode_attention_noalloc": (i32, [ctypes.POINTER(Layout), vp, vp, i64, vp, i32, vp, i32,
                                               vp, vp, vp, sz, vp, ctypes.POINTER(DecodeOpts), vp,
                                               vp]),
+    "starkv_diag_bounded_wait": (i32, [i32, vp, vp]),
     "starkv_last_error": (ctypes.c_char_p, []),
     "starkv_version": (i32, []),
 }

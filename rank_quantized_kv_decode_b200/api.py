@@ -92,8 +92,8 @@ def dequant(lay, cache, tok_seq, tok_pos, block_table, latents_out, status, stre
 
 def decode_attention(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rope_table, out, workspace,
                      status, max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
-                     stream=None) -> None:
-    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms)
+                     cta_group: int = 0, stream=None) -> None:
+    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms, cta_group)
     L.check(L.load().starkv_decode_attention(
         ctypes.byref(lay), _ptr(q), _ptr(cache),
         cache.numel() * cache.element_size() // lay.page_bytes, _ptr(block_table),
@@ -108,7 +108,7 @@ def decode_attention_noalloc(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rop
                              stream=None) -> None:
     """decode_attention with the library's built-in 16 MiB scratch instead of a workspace
     (for callers that cannot allocate device memory; see include/starkv.h)."""
-    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms)
+    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms, 0)
     L.check(L.load().starkv_decode_attention_noalloc(
         ctypes.byref(lay), _ptr(q), _ptr(cache),
         cache.numel() * cache.element_size() // lay.page_bytes, _ptr(block_table),
@@ -119,8 +119,8 @@ def decode_attention_noalloc(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rop
 
 def decode_partials(lay, q, cache, block_table, seq_lens, Bk_t, rope_table, workspace, status,
                     max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
-                    stream=None) -> None:
-    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms)
+                    cta_group: int = 0, stream=None) -> None:
+    opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms, cta_group)
     L.check(L.load().starkv_decode_partials(
         ctypes.byref(lay), _ptr(q), _ptr(cache),
         cache.numel() * cache.element_size() // lay.page_bytes, _ptr(block_table),
@@ -135,6 +135,11 @@ def decode_combine(lay, seq_lens, max_pages: int, Bv, workspace, out, stream=Non
         ctypes.byref(lay), _ptr(seq_lens), seq_lens.shape[0], max_pages, _ptr(Bv),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
         _stream(stream)), "starkv_decode_combine")
+
+
+def diag_bounded_wait(timeout_ms: int, status, stream=None) -> None:
+    L.check(L.load().starkv_diag_bounded_wait(timeout_ms, _ptr(status), _stream(stream)),
+            "starkv_diag_bounded_wait")
 
 
 def _bytes(n: int, device) -> torch.Tensor:

@@ -483,23 +483,33 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   p.NC = ncols >= 256 ? (fmt == STARKV_FMT_F32 ? 128 : 256) : ncols;
   p.n_chunks = ceil_div(ncols, p.NC);
   p.kb_count = ceil_div(c.key_rank * es, kKBytes);
+  // CTA pairs (one cluster per 256-token tile) for 16-bit operands and 256-column chunks
+  const int want_cg = opts ? opts->cta_group : 0;
+  if (want_cg < 0 || want_cg > 2) return fail(STARKV_ERR_INVALID_ARG, "cta_group must be 0, 1 or 2");
+  const bool pair_ok = fmt != STARKV_FMT_F32 && p.NC == 256 && info.sms >= 2;
+  if (want_cg == 2 && !pair_ok)
+    return fail(STARKV_ERR_UNSUPPORTED, "CTA pairs need bf16 or int8/int4 latents and 256-column chunks");
+  p.cta_group = (want_cg == 1 || !pair_ok) ? 1 : 2;
+  const int CG = p.cta_group;
   int grid_cap = info.sms;
   if (opts && opts->max_ctas > 0 && opts->max_ctas < grid_cap) grid_cap = opts->max_ctas;
+  grid_cap = std::max(CG, grid_cap / CG * CG);
+  const long long group_tiles = ceil_div(tiles_max, CG);
   int n_ranges = 1;
   if (opts && opts->n_ranges > 0) {
     n_ranges = std::min(opts->n_ranges, p.n_chunks);
   } else {
-    while (n_ranges < p.n_chunks && static_cast<long long>(batch) * tiles_max * n_ranges < 4LL * grid_cap)
+    while (n_ranges < p.n_chunks && batch * group_tiles * n_ranges < 4LL * (grid_cap / CG))
       n_ranges *= 2;
     n_ranges = std::min(n_ranges, p.n_chunks);
   }
   p.cpr = ceil_div(p.n_chunks, n_ranges);
   p.n_ranges = ceil_div(p.n_chunks, p.cpr);
-  const long long units = static_cast<long long>(tiles_max) * batch * p.n_ranges;
+  const long long units = group_tiles * batch * p.n_ranges;
   if (units > (1LL << 30)) return fail(STARKV_ERR_INVALID_ARG, "too many work units");
   p.total_units = static_cast<int>(units);
-  p.idesc = idesc_make(fmt == STARKV_FMT_F32 ? 2u : (fmt == STARKV_FMT_BF16 ? 1u : 0u), 128,
-                       static_cast<uint32_t>(p.NC));
+  p.idesc = idesc_make(fmt == STARKV_FMT_F32 ? 2u : (fmt == STARKV_FMT_BF16 ? 1u : 0u),
+                       static_cast<uint32_t>(128 * CG), static_cast<uint32_t>(p.NC));
   p.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   p.key = lat_desc(lay->seg[0]);
   int vmax = 0;
@@ -527,10 +537,10 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   // shared-memory plan: ring stages of (A k-block, B k-block), value buffers, small arrays
   const int HPW = 128 / d, QPW = HPW * p.G;
   p.vslot = (vmax + 127) / 128 * 128;
-  const size_t bstage = static_cast<size_t>(p.NC) * kKBytes;
+  const size_t bstage = static_cast<size_t>(p.NC / CG) * kKBytes;
   const size_t limit = std::min<size_t>(decode_smem_limit(), info.smem_optin);
   bool planned = false;
-  const int plans[][2] = {{4, 2}, {4, 1}, {3, 2}, {3, 1}, {2, 1}};
+  const int plans[][2] = {{6, 2}, {6, 1}, {5, 2}, {5, 1}, {4, 2}, {4, 1}, {3, 2}, {3, 1}, {2, 1}};
   for (const auto& pl : plans) {
     size_t off = 0;
     const int S = pl[0], NVB = pl[1];
@@ -593,11 +603,11 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
                                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(c.key_rank), static_cast<cuuint64_t>(ncols)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(c.key_rank) * es};
-    cuuint32_t box[2] = {ke, static_cast<cuuint32_t>(p.NC)};
+    cuuint32_t box[2] = {ke, static_cast<cuuint32_t>(p.NC / CG)};
     st = encode(&tmB, dt, 2, Bk_t, dims, strides, box);
     if (st != STARKV_OK) return st;
   }
-  grid = static_cast<int>(std::min<long long>(units, grid_cap));
+  grid = static_cast<int>(std::min<long long>(units * CG, grid_cap));
   return STARKV_OK;
 }
 
@@ -656,6 +666,20 @@ starkv_status starkv_decode_attention(const starkv_layout* lay, const void* q, c
   if (e != cudaSuccess) return cuda_fail(e, "decode split launch");
   e = launch_combine(p, s);
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  return STARKV_OK;
+}
+
+starkv_status starkv_diag_bounded_wait(int32_t timeout_ms, int32_t* dev_status,
+                                      starkv_stream_t stream) {
+  if (timeout_ms < 1 || timeout_ms > 10000)
+    return fail(STARKV_ERR_INVALID_ARG, "timeout_ms must be in [1, 10000]");
+  if (!dev_status) return fail(STARKV_ERR_INVALID_ARG, "dev_status is NULL");
+  DevInfo info;
+  starkv_status st = current_device(info);
+  if (st != STARKV_OK) return st;
+  cudaError_t e = launch_bounded_wait(dev_status, static_cast<unsigned long long>(timeout_ms) * 1000000ull,
+                                      reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bounded-wait diagnostic launch");
   return STARKV_OK;
 }
 

@@ -34,12 +34,18 @@ struct Unit {
   __device__ __forceinline__ int page(int half) const { return half ? page1 : page0; }
 };
 
-// Same answer in every role: the pipelines of all warps walk the same unit sequence.
-__device__ __forceinline__ bool get_unit(const DecodeParams& p, int u, Unit& U, bool flag) {
+// Same answer in every role: the pipelines of all warps walk the same unit sequence.  With a
+// CTA pair (CG = 2) a unit covers a 256-token tile; CTA ``crank`` owns its 128-token half.
+// A unit exists when its first token is inside the sequence; the half may still be empty
+// (nvalid = 0, no pages).
+template <int CG>
+__device__ __forceinline__ bool get_unit(const DecodeParams& p, int u, Unit& U, bool flag,
+                                         int crank) {
   const int rg = u % p.n_ranges;
   const int rest = u / p.n_ranges;
   U.b = rest % p.batch;
-  U.tile = rest / p.batch;
+  const int group_tile = rest / p.batch;
+  U.tile = group_tile * CG + crank;
   int L = p.seq_lens[U.b];
   const int cap = p.max_pages * kPage;
   if (L > cap || L < 0) {
@@ -47,11 +53,11 @@ __device__ __forceinline__ bool get_unit(const DecodeParams& p, int u, Unit& U, 
     L = L < 0 ? 0 : cap;
   }
   U.L = L;
-  if (U.tile * kTile >= L) return false;
+  if (group_tile * CG * kTile >= L) return false;
   U.c0 = rg * p.cpr;
   U.c1 = min(U.c0 + p.cpr, p.n_chunks);
   if (U.c0 >= U.c1) return false;
-  U.nvalid = min(kTile, L - U.tile * kTile);
+  U.nvalid = max(0, min(kTile, L - U.tile * kTile));
   int pgs[2];
 #pragma unroll
   for (int pp = 0; pp < 2; ++pp) {
@@ -191,7 +197,7 @@ __device__ __forceinline__ float qload(const void* q, long long idx) {
 
 }  // namespace
 
-template <int FMT, int HD, int G>
+template <int FMT, int HD, int G, int CG>
 __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams p,
                         const __grid_constant__ CUtensorMap tmA,
@@ -204,9 +210,15 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  static_assert(CG == 1 || !Fmt<FMT>::kSplit, "fp32 latents use single-CTA tiles");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages, NVB = p.nvb;
-  const uint32_t bstage = static_cast<uint32_t>(p.NC) * kKBytes;
+  // CTA pair: this CTA's rank, and the pair's unit stream
+  const int crank = CG == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+  const bool leader = crank == 0;
+  const int unit0 = blockIdx.x / CG, unit_step = gridDim.x / CG;
+  // this CTA's B rows per k-block: the whole chunk, or its half of it in a pair
+  const uint32_t bstage = static_cast<uint32_t>(p.NC / CG) * kKBytes;
   // stage strides: the split format keeps hi and lo copies of both operands
   const uint32_t astride = F::kSplit ? 2 * kAStage : kAStage;
   const uint32_t bstride = F::kSplit ? 2 * bstage : bstage;
@@ -226,14 +238,16 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   if (threadIdx.x == 0) {
+    // a pair's full barriers (in the leader) count both CTAs' producers and dequantisers;
+    // its accumulator-empty barriers count the epilogue warps of both CTAs
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar(B_FULL + s), F::kFullCount);
+      mbar_init(bar(B_FULL + s), CG == 1 ? F::kFullCount : (F::kTmaA ? 2 : 10));
       mbar_init(bar(B_EMPTY + s), 1);
       mbar_init(bar(B_RAW + s), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(B_ACCF + a), 1);
-      mbar_init(bar(B_ACCE + a), 8);
+      mbar_init(bar(B_ACCE + a), 8 * CG);
     }
     for (int v = 0; v < NVB; ++v) {
       mbar_init(bar(B_VF + v), 1);
@@ -248,13 +262,23 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     if constexpr (F::kTmaA) prefetch_tmap(&tmA);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(misc), 512);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(smem_u32(misc), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(misc), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2)
+    cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA arrive or copy
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
+  // the pair's MMA-side barriers live in the leader CTA
+  auto leader_bar = [&](int i) { return CG == 2 ? mapa_shared(bar(i), 0) : bar(i); };
   WaitCtl wc{reinterpret_cast<volatile int*>(misc + 1), p.status, p.timeout_ns};
 
   if (warp == 0) {
@@ -263,44 +287,65 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.total_units; u += unit_step) {
         Unit U;
-        if (!get_unit(p, u, U, true)) continue;
+        if (!get_unit<CG>(p, u, U, true, crank)) continue;
         for (int c = U.c0; ok && c < U.c1; ++c) {
           for (int kb = 0; kb < p.kb_count; ++kb) {
             if (!wait_bounded(bar(B_EMPTY + stage), phase ^ 1u, wc)) { ok = false; break; }
             uint32_t bytes = bstage;
             if constexpr (F::kTmaA)
               bytes += (U.page0 >= 0 ? 8192u : 0u) + (U.page1 >= 0 ? 8192u : 0u);
-            // the split format lands raw fp32 tiles that the converters turn into hi/lo
-            const uint32_t fb = bar((F::kSplit ? B_RAW : B_FULL) + stage);
-            mbar_arrive_expect_tx(fb, bytes);
-            if constexpr (F::kTmaA) {
-              const uint32_t da = smem_u32(sA + stage * astride);
-              if (U.page0 >= 0) tma_load_3d(da, &tmA, fb, kb * F::kKElems, 0, U.page0);
-              if (U.page1 >= 0) tma_load_3d(da + 8192, &tmA, fb, kb * F::kKElems, 0, U.page1);
+            const uint32_t da = smem_u32(sA + stage * astride);
+            const uint32_t db = smem_u32(sB + stage * bstride);
+            const int brow = c * p.NC + crank * (p.NC / CG);
+            if constexpr (CG == 2) {
+              // both CTAs' bytes complete the leader's full barrier
+              const uint32_t fb = leader_bar(B_FULL + stage);
+              mbar_arrive_expect_tx_cluster(fb, bytes);
+              if constexpr (F::kTmaA) {
+                if (U.page0 >= 0) tma_load_3d_pair(da, &tmA, fb, kb * F::kKElems, 0, U.page0);
+                if (U.page1 >= 0) tma_load_3d_pair(da + 8192, &tmA, fb, kb * F::kKElems, 0, U.page1);
+              }
+              tma_load_2d_pair(db, &tmB, fb, kb * F::kKElems, brow);
+            } else {
+              // the split format lands raw fp32 tiles that the converters turn into hi/lo
+              const uint32_t fb = bar((F::kSplit ? B_RAW : B_FULL) + stage);
+              mbar_arrive_expect_tx(fb, bytes);
+              if constexpr (F::kTmaA) {
+                if (U.page0 >= 0) tma_load_3d(da, &tmA, fb, kb * F::kKElems, 0, U.page0);
+                if (U.page1 >= 0) tma_load_3d(da + 8192, &tmA, fb, kb * F::kKElems, 0, U.page1);
+              }
+              tma_load_2d(db, &tmB, fb, kb * F::kKElems, brow);
             }
-            tma_load_2d(smem_u32(sB + stage * bstride), &tmB, fb, kb * F::kKElems, c * p.NC);
             issued |= 1u << stage;
             last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
             if (++stage == S) { stage = 0; phase ^= 1u; }
           }
         }
       }
-      // every copy this thread started has landed before the CTA may exit
-      for (int s = 0; s < S; ++s)
-        if (issued & (1u << s))
-          wait_drain(bar((F::kSplit ? B_RAW : B_FULL) + s), (last_phase >> s) & 1u, p.timeout_ns);
+      // every copy this thread started has landed before the CTA may exit: the leader's
+      // full barriers see both CTAs' bytes; after an abort the other CTA of a pair, which
+      // cannot wait on them, gives its copies a fixed grace period instead
+      if (CG == 1 || leader) {
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s))
+            wait_drain(bar((F::kSplit ? B_RAW : B_FULL) + s), (last_phase >> s) & 1u, p.timeout_ns);
+      } else if (!ok) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0, ab = 0;
       uint32_t phase = 0, aph = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.total_units; u += unit_step) {
         Unit U;
-        if (!get_unit(p, u, U, false)) continue;
+        if (!get_unit<CG>(p, u, U, false, crank)) continue;
         for (int c = U.c0; ok && c < U.c1; ++c) {
           if (!wait_bounded(bar(B_ACCE + ab), aph ^ 1u, wc)) { ok = false; break; }
           tc_fence_after();
@@ -312,24 +357,38 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             const uint64_t db = desc_sw128(smem_u32(sB + stage * bstride));
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              umma<F::kKind>(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
-              if constexpr (F::kSplit) {
-                const uint64_t dal = desc_sw128(smem_u32(sA + stage * astride + kAStage));
-                const uint64_t dbl = desc_sw128(smem_u32(sB + stage * bstride + bstage));
-                umma<F::kKind>(d_tmem, da + 2 * k, dbl + 2 * k, p.idesc, 1u);
-                umma<F::kKind>(d_tmem, dal + 2 * k, db + 2 * k, p.idesc, 1u);
+              if constexpr (CG == 2) {
+                umma_f16_pair(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
+              } else {
+                umma<F::kKind>(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
+                if constexpr (F::kSplit) {
+                  const uint64_t dal = desc_sw128(smem_u32(sA + stage * astride + kAStage));
+                  const uint64_t dbl = desc_sw128(smem_u32(sB + stage * bstride + bstage));
+                  umma<F::kKind>(d_tmem, da + 2 * k, dbl + 2 * k, p.idesc, 1u);
+                  umma<F::kKind>(d_tmem, dal + 2 * k, db + 2 * k, p.idesc, 1u);
+                }
               }
             }
-            umma_commit(bar(B_EMPTY + stage));
+            // the stage is free in both CTAs once these MMAs have read it
+            if constexpr (CG == 2)
+              umma_commit_pair(bar(B_EMPTY + stage), 3);
+            else
+              umma_commit(bar(B_EMPTY + stage));
             if (++stage == S) { stage = 0; phase ^= 1u; }
           }
           if (!ok) break;
-          umma_commit(bar(B_ACCF + ab));
+          if constexpr (CG == 2)
+            umma_commit_pair(bar(B_ACCF + ab), 3);
+          else
+            umma_commit(bar(B_ACCF + ab));
           ab ^= 1;
           if (ab == 0) aph ^= 1u;
         }
       }
-      umma_commit(bar(B_TD));
+      if constexpr (CG == 2)
+        umma_commit_pair(bar(B_TD), 1);
+      else
+        umma_commit(bar(B_TD));
       wait_drain(bar(B_TD), 0, p.timeout_ns);
     }
     __syncwarp();
@@ -339,9 +398,9 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       int vs = 0;
       uint32_t vph = 0, issued = 0, last_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.total_units; u += unit_step) {
         Unit U;
-        if (!get_unit(p, u, U, false)) continue;
+        if (!get_unit<CG>(p, u, U, false, crank)) continue;
         for (int c = U.c0; c < U.c1; ++c) {
           if (!wait_bounded(bar(B_VE + vs), vph ^ 1u, wc)) { ok = false; break; }
           const uint32_t nbytes = static_cast<uint32_t>(p.vchunk_bytes[c]);
@@ -389,16 +448,17 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     bool stop = false;
     // head slots of this warpgroup that belong to a chunk (NC may be 128: then only WG 0)
     const int wg_slots = max(0, min(HPW, p.NC / HD - wg * HPW));
-    for (int u = blockIdx.x; !stop && u < p.total_units; u += gridDim.x) {
+    for (int u = unit0; !stop && u < p.total_units; u += unit_step) {
       Unit U;
-      if (!get_unit(p, u, U, false)) continue;
+      if (!get_unit<CG>(p, u, U, false, crank)) continue;
       const int T = U.L - 1;  // position of the decode query
+      const bool has_rows = U.nvalid > 0;  // the pair's second half may lie past the end
       const bool rv = row < U.nvalid && U.page(row >> 6) >= 0;
       for (int c = U.c0; c < U.c1; ++c) {
         const int g_first = c * (p.NC / HD) + wg * HPW;
         // (1) rotated, scaled queries of this warpgroup's heads; the tile's start angles
         for (int j = row; j < HALF; j += 128) {
-          const float2 bs = basetab[U.tile * HALF + j];
+          const float2 bs = basetab[min(U.tile, p.rope_tiles - 1) * HALF + j];
           phi_s[j] = atan2f(bs.y, bs.x);
         }
         for (int idx = row; idx < QPW * HALF; idx += 128) {
@@ -469,7 +529,12 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_ACCE + ab));
+        if (lane == 0) {
+          if (CG == 2 && !leader)
+            mbar_arrive_cluster(leader_bar(B_ACCE + ab));
+          else
+            mbar_arrive(bar(B_ACCE + ab));
+        }
         ab ^= 1;
         if (ab == 0) aph ^= 1u;
         // (4) tile-local softmax statistics (log2 domain: scores carry log2(e)/sqrt(d))
@@ -499,7 +564,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
 #pragma unroll
         for (int hs = 0; hs < HPW; ++hs) {
           const int g = g_first + hs;
-          if (g >= p.Hkv || hs >= wg_slots) continue;
+          if (g >= p.Hkv || hs >= wg_slots || !has_rows) continue;
           const LatDesc& vd = p.vh[g];
           if (row < vd.rank) {
             float a[G];
@@ -548,9 +613,9 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.total_units; u += unit_step) {
         Unit U;
-        if (!get_unit(p, u, U, false)) continue;
+        if (!get_unit<CG>(p, u, U, false, crank)) continue;
         for (int c = U.c0; ok && c < U.c1; ++c) {
           for (int kb = 0; kb < p.kb_count; ++kb) {
             if (!__all_sync(0xffffffffu, wait_bounded(bar(B_RAW + stage), phase, wc))) {
@@ -577,9 +642,9 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.total_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.total_units; u += unit_step) {
         Unit U;
-        if (!get_unit(p, u, U, false)) continue;
+        if (!get_unit<CG>(p, u, U, false, crank)) continue;
         for (int c = U.c0; ok && c < U.c1; ++c) {
           for (int kb = 0; kb < p.kb_count; ++kb) {
             // warp-uniform decision (the __syncwarp below needs every lane)
@@ -597,7 +662,12 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_FULL + stage));
+            if (lane == 0) {
+              if constexpr (CG == 2)
+                mbar_arrive_cluster(leader_bar(B_FULL + stage));
+              else
+                mbar_arrive(bar(B_FULL + stage));
+            }
             if (++stage == S) { stage = 0; phase ^= 1u; }
           }
         }
@@ -606,9 +676,16 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if constexpr (CG == 2) {
+    // neither CTA leaves while the pair's MMAs may still read its shared memory or TMEM
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, 512);
+  } else {
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+  }
 }
 
 // --------------------------------------------------------------------------- combine
@@ -677,44 +754,62 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
 }
 
 // --------------------------------------------------------------------------- launchers
-template <int FMT, int HD, int G>
+template <int FMT, int HD, int G, int CG>
 static cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tmA,
                               const CUtensorMap& tmB, int grid, cudaStream_t s) {
-  auto kern = decode_split_kernel<FMT, HD, G>;
+  auto kern = decode_split_kernel<FMT, HD, G, CG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(p.smem_bytes));
   if (e != cudaSuccess) return e;
-  kern<<<grid, Fmt<FMT>::kWarps * 32, p.smem_bytes, s>>>(p, tmA, tmB);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(Fmt<FMT>::kWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, tmA, tmB);
 }
 
-template <int FMT, int HD>
+template <int FMT, int HD, int CG>
 static cudaError_t launch_g(int G, const DecodeParams& p, const CUtensorMap& tmA,
                             const CUtensorMap& tmB, int grid, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_one<FMT, HD, 1>(p, tmA, tmB, grid, s);
-    case 2: return launch_one<FMT, HD, 2>(p, tmA, tmB, grid, s);
-    case 4: return launch_one<FMT, HD, 4>(p, tmA, tmB, grid, s);
-    case 8: return launch_one<FMT, HD, 8>(p, tmA, tmB, grid, s);
+    case 1: return launch_one<FMT, HD, 1, CG>(p, tmA, tmB, grid, s);
+    case 2: return launch_one<FMT, HD, 2, CG>(p, tmA, tmB, grid, s);
+    case 4: return launch_one<FMT, HD, 4, CG>(p, tmA, tmB, grid, s);
+    case 8: return launch_one<FMT, HD, 8, CG>(p, tmA, tmB, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int FMT>
+template <int FMT, int CG>
 static cudaError_t launch_hd(int hd, int G, const DecodeParams& p, const CUtensorMap& tmA,
                              const CUtensorMap& tmB, int grid, cudaStream_t s) {
-  if (hd == 64) return launch_g<FMT, 64>(G, p, tmA, tmB, grid, s);
-  if (hd == 128) return launch_g<FMT, 128>(G, p, tmA, tmB, grid, s);
+  if (hd == 64) return launch_g<FMT, 64, CG>(G, p, tmA, tmB, grid, s);
+  if (hd == 128) return launch_g<FMT, 128, CG>(G, p, tmA, tmB, grid, s);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
                           const CUtensorMap& tmA, const CUtensorMap& tmB, int grid,
                           cudaStream_t s) {
+  if (p.cta_group == 2) {
+    switch (fmt) {
+      case STARKV_FMT_BF16: return launch_hd<FMT_BF16, 2>(head_dim, G, p, tmA, tmB, grid, s);
+      case STARKV_FMT_MIXED: return launch_hd<FMT_MIXED, 2>(head_dim, G, p, tmA, tmB, grid, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (fmt) {
-    case STARKV_FMT_F32: return launch_hd<FMT_F32>(head_dim, G, p, tmA, tmB, grid, s);
-    case STARKV_FMT_BF16: return launch_hd<FMT_BF16>(head_dim, G, p, tmA, tmB, grid, s);
-    case STARKV_FMT_MIXED: return launch_hd<FMT_MIXED>(head_dim, G, p, tmA, tmB, grid, s);
+    case STARKV_FMT_F32: return launch_hd<FMT_F32, 1>(head_dim, G, p, tmA, tmB, grid, s);
+    case STARKV_FMT_BF16: return launch_hd<FMT_BF16, 1>(head_dim, G, p, tmA, tmB, grid, s);
+    case STARKV_FMT_MIXED: return launch_hd<FMT_MIXED, 1>(head_dim, G, p, tmA, tmB, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

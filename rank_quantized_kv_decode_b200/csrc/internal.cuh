@@ -61,6 +61,7 @@ struct DecodeParams {
   unsigned long long timeout_ns;
   int H, Hkv, G, d, rk, key_rank_cols;
   int NC, n_chunks, n_ranges, cpr, kb_count, total_units;
+  int cta_group;  // 1: one CTA per 128-token tile; 2: a CTA pair per 256-token tile
   uint32_t idesc;
   float qscale;  // log2(e) / sqrt(d)
   // dynamic shared-memory plan (offsets from the 1024-aligned base)
@@ -84,6 +85,7 @@ cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
                           const CUtensorMap& tmA, const CUtensorMap& tmB, int grid,
                           cudaStream_t s);
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_bounded_wait(int* status, unsigned long long timeout_ns, cudaStream_t s);
 size_t decode_smem_limit();
 
 struct ProjParams {

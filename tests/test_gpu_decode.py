@@ -55,17 +55,27 @@ def test_decode_matches_oracle(index):
 
 
 @pytest.mark.parametrize("index", [2, 4])
-@pytest.mark.parametrize("max_ctas,n_ranges", [(1, 1), (7, 2), (0, 4), (3, 0)])
-def test_launch_shape_does_not_change_result(index, max_ctas, n_ranges):
+@pytest.mark.parametrize("cta_group", [1, 2])
+@pytest.mark.parametrize("max_ctas,n_ranges", [(2, 1), (8, 2), (0, 4), (6, 0)])
+def test_launch_shape_does_not_change_result(index, cta_group, max_ctas, n_ranges):
     wl = built(index)
-    W.decode(wl)
+    W.decode(wl, cta_group=cta_group)
     torch.cuda.synchronize()
     base = wl.out.clone()
-    W.decode(wl, max_ctas=max_ctas, n_ranges=n_ranges)
+    W.decode(wl, cta_group=cta_group, max_ctas=max_ctas, n_ranges=n_ranges)
     torch.cuda.synchronize()
     assert wl.lc.status.item() == 0
     # each tile's partial is computed the same way whatever the grid: bit-identical
     assert torch.equal(base, wl.out)
+
+
+@pytest.mark.parametrize("index", [2, 3, 4, 5])
+@pytest.mark.parametrize("cta_group", [1, 2])
+def test_single_and_paired_ctas_match_oracle(index, cta_group):
+    wl = built(index)
+    W.decode(wl, cta_group=cta_group)
+    torch.cuda.synchronize()
+    check_all(index, wl)
 
 
 @pytest.mark.parametrize("index", [1, 4])
