@@ -535,7 +535,6 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   for (int g = 0; g < c.n_kv_heads; ++g) p.vh[g] = lat_desc(lay->seg[1 + g]);
 
   // shared-memory plan: ring stages of (A k-block, B k-block), value buffers, small arrays
-  const int HPW = 128 / d, QPW = HPW * p.G;
   p.vslot = (vmax + 127) / 128 * 128;
   const size_t bstage = static_cast<size_t>(p.NC / CG) * kKBytes;
   const size_t limit = std::min<size_t>(decode_smem_limit(), info.smem_optin);
@@ -550,15 +549,21 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     off += S * split * bstage;
     const size_t off_v = off;
     off += static_cast<size_t>(NVB) * 2 * p.vslot;
+    const size_t QPC = static_cast<size_t>(256 / d) * p.G;  // query heads of a full chunk
     const size_t off_q = off;
-    off += 2 * static_cast<size_t>(QPW) * d * 4;
+    off += QPC * d * 4;
     const size_t off_p = off;
-    off += 2 * static_cast<size_t>(QPW) * kTile * 4;
+    off += QPC * kTile * 4;
+    const size_t off_part = off;
+    off += 2 * QPC * kTile * 4;
     const size_t off_red = off;
-    off += 2 * 2 * static_cast<size_t>(QPW) * 4 * 4;
+    off += 2 * 2 * QPC * 4 * 4;
     off = (off + 15) / 16 * 16;
     const size_t off_ang = off;
-    off += 2 * 2 * static_cast<size_t>(d / 2) * 4;
+    off += 2 * static_cast<size_t>(d / 2) * 4;
+    const size_t off_pv = off;
+    off += 2 * static_cast<size_t>(p.G) * kTile * 4;
+    off = (off + 7) / 8 * 8;
     const size_t off_bar = off;
     off += (3 * S + 4 + 2 * NVB + 1) * 8 + 16;
     // alignment slack of the dynamic base; at least 120 KB so that one CTA occupies an SM
@@ -571,8 +576,10 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
       p.off_v = static_cast<uint32_t>(off_v);
       p.off_q = static_cast<uint32_t>(off_q);
       p.off_p = static_cast<uint32_t>(off_p);
+      p.off_part = static_cast<uint32_t>(off_part);
       p.off_red = static_cast<uint32_t>(off_red);
       p.off_ang = static_cast<uint32_t>(off_ang);
+      p.off_pv = static_cast<uint32_t>(off_pv);
       p.off_bar = static_cast<uint32_t>(off_bar);
       p.smem_bytes = static_cast<uint32_t>(total);
       planned = true;

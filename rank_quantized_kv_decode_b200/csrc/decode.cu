@@ -203,8 +203,6 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
                         const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB) {
   using F = Fmt<FMT>;
-  constexpr int HPW = 128 / HD;  // KV heads per epilogue warpgroup
-  constexpr int QPW = HPW * G;   // query heads per epilogue warpgroup
   constexpr int HALF = HD / 2;
 
   extern __shared__ uint8_t smem_raw[];
@@ -226,10 +224,13 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + p.off_b;
   uint8_t* sV = smem + p.off_v;
-  float* sQ = reinterpret_cast<float*>(smem + p.off_q);    // [2][QPW][HD]
-  float* sP = reinterpret_cast<float*>(smem + p.off_p);    // [2][QPW][128]
-  float* sRed = reinterpret_cast<float*>(smem + p.off_red);  // [2][2][QPW][4]
-  float* sAng = reinterpret_cast<float*>(smem + p.off_ang);  // [2][2][HALF]: theta_j, tile angle
+  // epilogue scratch; QPC = query heads of a 256-column chunk
+  float* sQ = reinterpret_cast<float*>(smem + p.off_q);        // [QPC][HD] rotated queries
+  float* sP = reinterpret_cast<float*>(smem + p.off_p);        // [QPC][128] probabilities
+  float* sPart = reinterpret_cast<float*>(smem + p.off_part);  // [2][QPC][128] partial scores
+  float* sRed = reinterpret_cast<float*>(smem + p.off_red);    // [2][2][QPC][4] reductions
+  float* sAng = reinterpret_cast<float*>(smem + p.off_ang);    // [2][HALF] theta_j, phi_j
+  float* sPV = reinterpret_cast<float*>(smem + p.off_pv);      // [2][G][128] P.C_v partials
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   const int B_FULL = 0, B_EMPTY = S, B_RAW = 2 * S, B_ACCF = 3 * S, B_ACCE = 3 * S + 2,
             B_VF = 3 * S + 4, B_VE = 3 * S + 4 + NVB, B_TD = 3 * S + 4 + 2 * NVB;
@@ -302,7 +303,10 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             if constexpr (CG == 2) {
               // both CTAs' bytes complete the leader's full barrier
               const uint32_t fb = leader_bar(B_FULL + stage);
-              mbar_arrive_expect_tx_cluster(fb, bytes);
+              if (leader)
+                mbar_arrive_expect_tx(bar(B_FULL + stage), bytes);
+              else
+                mbar_arrive_expect_tx_cluster(fb, bytes);
               if constexpr (F::kTmaA) {
                 if (U.page0 >= 0) tma_load_3d_pair(da, &tmA, fb, kb * F::kKElems, 0, U.page0);
                 if (U.page1 >= 0) tma_load_3d_pair(da + 8192, &tmA, fb, kb * F::kKElems, 0, U.page1);
@@ -422,111 +426,131 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     }
   } else if (warp >= 4 && warp < 12) {
     // ---------------------------------------------------------------- epilogue warpgroups
+    // Thread = token row (its TMEM lane).  Scores: warpgroup w rotates and dots the RoPE
+    // pairs [w*JW, (w+1)*JW) of every KV head of the chunk, so each angle's sine and cosine is
+    // computed once per row; the two partial scores meet in shared memory.  Softmax and the
+    // latent P.C_v: warpgroup w owns half of the chunk's KV heads.
+    constexpr int HPC = 256 / HD;  // KV heads in a full 256-column chunk
+    constexpr int QPC = HPC * G;   // their query heads
+    constexpr int JW = HALF / 2;   // RoPE pairs per warpgroup
+    constexpr int JG = 8;          // pairs per step (one 8-column TMEM load per half)
+    constexpr int NSTEP = (JW / JG) * HPC;
     const int wg = (warp - 4) >> 2;
     const int quad = warp & 3;          // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;   // token row in the tile == thread index in the WG
+    const int et = wg * 128 + row;      // thread index over both warpgroups
+    const int hpc = p.NC / HD;          // KV heads per chunk in this launch (NC may be 128)
+    const int own_n = (hpc + 1) / 2;    // head slots whose softmax this warpgroup does
+    const int own0 = wg * own_n;
     const float2* fine = p.rope;
     const float2* basetab = p.rope + kTile * HALF;
-    // RoPE angles of this warpgroup: theta_j (fixed) and the tile-start angle phi_j, both
-    // recovered from the fp64-built table; a row's angle phi_j + r*theta_j stays below
-    // pi + 128, where the SFU sine/cosine error is ~1e-5 rad -- no per-element table reads
-    float* theta_s = sAng + wg * 2 * HALF;
-    float* phi_s = theta_s + HALF;
-    for (int j = row; j < HALF; j += 128) {
+    // RoPE angles: theta_j (fixed) and the tile-start angle phi_j, both recovered from the
+    // fp64-built table; a row's angle phi_j + r*theta_j stays below pi + 128, where the SFU
+    // sine/cosine error is ~1e-5 rad -- no per-element table reads
+    float* theta_s = sAng;
+    float* phi_s = sAng + HALF;
+    float* red = sRed + wg * 2 * QPC * 4;
+    float* pv = sPV + wg * G * kTile;
+    int* s_stop = reinterpret_cast<int*>(misc + 2);
+    for (int j = et; j < HALF; j += 256) {
       const float2 f1 = fine[HALF + j];  // row 1: angle theta_j
       theta_s[j] = atan2f(f1.y, f1.x);
     }
     const float rowf = static_cast<float>(row);
-    float* q_s = sQ + wg * QPW * HD;
-    float* p_s = sP + wg * QPW * kTile;
-    float* red = sRed + wg * 2 * QPW * 4;
-    int* s_stop = reinterpret_cast<int*>(misc + 2);  // [2] per-warpgroup snapshot of abort
     int ab = 0, vs = 0;
     uint32_t aph = 0, vph = 0;
-    // Control flow of a warpgroup only changes on a snapshot every thread reads after a
-    // named barrier, so no thread can leave while the others wait at a barrier.
+    // Control flow of the epilogue only changes on a snapshot every thread reads after a
+    // barrier of both warpgroups, so no thread leaves while others wait at a barrier.
     bool stop = false;
-    // head slots of this warpgroup that belong to a chunk (NC may be 128: then only WG 0)
-    const int wg_slots = max(0, min(HPW, p.NC / HD - wg * HPW));
     for (int u = unit0; !stop && u < p.total_units; u += unit_step) {
       Unit U;
       if (!get_unit<CG>(p, u, U, false, crank)) continue;
       const int T = U.L - 1;  // position of the decode query
-      const bool has_rows = U.nvalid > 0;  // the pair's second half may lie past the end
       const bool rv = row < U.nvalid && U.page(row >> 6) >= 0;
+      const bool has_rows = U.nvalid > 0;  // a pair's second half may lie past the end
       for (int c = U.c0; c < U.c1; ++c) {
-        const int g_first = c * (p.NC / HD) + wg * HPW;
-        // (1) rotated, scaled queries of this warpgroup's heads; the tile's start angles
-        for (int j = row; j < HALF; j += 128) {
-          const float2 bs = basetab[min(U.tile, p.rope_tiles - 1) * HALF + j];
-          phi_s[j] = atan2f(bs.y, bs.x);
-        }
-        for (int idx = row; idx < QPW * HALF; idx += 128) {
+        const int g0 = c * hpc;  // first KV head of the chunk
+        // (1) rotated, scaled queries of every head of the chunk; the tile's start angles
+        for (int idx = et; idx < hpc * G * HALF; idx += 256) {
           const int hq = idx / HALF, j = idx % HALF;
-          const int g = g_first + hq / G;
-          if (g >= p.Hkv || hq / G >= wg_slots) continue;
+          const int g = g0 + hq / G;
+          if (g >= p.Hkv) continue;
           const int h = g * G + hq % G;
           const long long qb = ((long long)U.b * p.H + h) * HD;
           const float x0 = qload<FMT>(p.q, qb + j), x1 = qload<FMT>(p.q, qb + j + HALF);
           const float2 bs = basetab[(T >> 7) * HALF + j], f = fine[(T & 127) * HALF + j];
           const float cs = bs.x * f.x - bs.y * f.y, sn = bs.y * f.x + bs.x * f.y;
-          q_s[hq * HD + j] = (x0 * cs - x1 * sn) * p.qscale;
-          q_s[hq * HD + j + HALF] = (x1 * cs + x0 * sn) * p.qscale;
+          sQ[hq * HD + j] = (x0 * cs - x1 * sn) * p.qscale;
+          sQ[hq * HD + j + HALF] = (x1 * cs + x0 * sn) * p.qscale;
         }
-        named_bar(1 + wg, 128);
+        for (int j = et; j < HALF; j += 256) {
+          const float2 bs = basetab[min(U.tile, p.rope_tiles - 1) * HALF + j];
+          phi_s[j] = atan2f(bs.y, bs.x);
+        }
+        named_bar(1, 256);
         // (2) accumulator of this chunk (on a timeout the data is garbage and the snapshot
         // below ends the loop)
         wait_bounded(bar(B_ACCF + ab), aph, wc);
         tc_fence_after();
-        // (3) RoPE on the reconstructed key row, scores of the GQA group
-        float sc[QPW];
+        // (3) partial scores over this warpgroup's pairs, every head; TMEM loads pipelined
+        float sc[QPC];
 #pragma unroll
-        for (int hs = 0; hs < HPW; ++hs) {
-          float acc[G];
+        for (int i = 0; i < QPC; ++i) sc[i] = 0.f;
+        {
+          const uint32_t tbase = tmem + static_cast<uint32_t>(ab * 256) +
+                                 (static_cast<uint32_t>(quad * 32) << 16);
+          const int jw0 = wg * JW;
+          uint32_t kb[2][16];
+          float cs[JG], sn[JG];
+          tmem_ld8x2(tbase + jw0, tbase + jw0 + HALF, kb[0]);
 #pragma unroll
-          for (int gq = 0; gq < G; ++gq) acc[gq] = 0.f;
-          if (g_first + hs < p.Hkv && hs < wg_slots) {
-            const uint32_t taddr = tmem + static_cast<uint32_t>(ab * 256 + wg * 128 + hs * HD) +
-                                   (static_cast<uint32_t>(quad * 32) << 16);
-#pragma unroll 1
-            for (int jj = 0; jj < HALF; jj += 16) {
-              float klo[16], khi[16];
-              tmem_ld16x2_wait(taddr + jj, taddr + HALF + jj, klo, khi);
+          for (int st = 0; st < NSTEP; ++st) {
+            const int jg = st / HPC, sl = st % HPC;
+            const int j0 = jw0 + jg * JG;
+            tmem_wait_regs16(kb[st & 1]);
+            if (st + 1 < NSTEP) {
+              const int jn = jw0 + ((st + 1) / HPC) * JG, sn1 = (st + 1) % HPC;
+              tmem_ld8x2(tbase + sn1 * HD + jn, tbase + sn1 * HD + jn + HALF, kb[(st + 1) & 1]);
+            }
+            if (sl == 0) {
 #pragma unroll
-              for (int j4 = 0; j4 < 4; ++j4) {
-                const int j0 = jj + 4 * j4;
-                const float4 th = *reinterpret_cast<const float4*>(theta_s + j0);
-                const float4 ph = *reinterpret_cast<const float4*>(phi_s + j0);
-                float cs[4], sn[4];
-                __sincosf(fmaf(rowf, th.x, ph.x), &sn[0], &cs[0]);
-                __sincosf(fmaf(rowf, th.y, ph.y), &sn[1], &cs[1]);
-                __sincosf(fmaf(rowf, th.z, ph.z), &sn[2], &cs[2]);
-                __sincosf(fmaf(rowf, th.w, ph.w), &sn[3], &cs[3]);
-                float k0[4], k1[4];
+              for (int e = 0; e < JG; e += 4) {
+                const float4 th = *reinterpret_cast<const float4*>(theta_s + j0 + e);
+                const float4 ph = *reinterpret_cast<const float4*>(phi_s + j0 + e);
+                __sincosf(fmaf(rowf, th.x, ph.x), &sn[e + 0], &cs[e + 0]);
+                __sincosf(fmaf(rowf, th.y, ph.y), &sn[e + 1], &cs[e + 1]);
+                __sincosf(fmaf(rowf, th.z, ph.z), &sn[e + 2], &cs[e + 2]);
+                __sincosf(fmaf(rowf, th.w, ph.w), &sn[e + 3], &cs[e + 3]);
+              }
+            }
+            if (sl < hpc) {
+              float k0[JG], k1[JG];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float a = klo[4 * j4 + e], b = khi[4 * j4 + e];
-                  k0[e] = a * cs[e] - b * sn[e];
-                  k1[e] = b * cs[e] + a * sn[e];
+              for (int e = 0; e < JG; ++e) {
+                const float a = __uint_as_float(kb[st & 1][e]);
+                const float b = __uint_as_float(kb[st & 1][JG + e]);
+                k0[e] = a * cs[e] - b * sn[e];
+                k1[e] = b * cs[e] + a * sn[e];
+              }
+#pragma unroll
+              for (int gq = 0; gq < G; ++gq) {
+                const float* qq = sQ + (sl * G + gq) * HD + j0;
+                float t = sc[sl * G + gq];
+#pragma unroll
+                for (int e = 0; e < JG; e += 4) {
+                  const float4 qa = *reinterpret_cast<const float4*>(qq + e);
+                  const float4 qb = *reinterpret_cast<const float4*>(qq + HALF + e);
+                  t = fmaf(k0[e + 0], qa.x, t); t = fmaf(k1[e + 0], qb.x, t);
+                  t = fmaf(k0[e + 1], qa.y, t); t = fmaf(k1[e + 1], qb.y, t);
+                  t = fmaf(k0[e + 2], qa.z, t); t = fmaf(k1[e + 2], qb.z, t);
+                  t = fmaf(k0[e + 3], qa.w, t); t = fmaf(k1[e + 3], qb.w, t);
                 }
-#pragma unroll
-                for (int gq = 0; gq < G; ++gq) {
-                  const float* qq = q_s + (hs * G + gq) * HD + j0;
-                  const float4 qa = *reinterpret_cast<const float4*>(qq);
-                  const float4 qb = *reinterpret_cast<const float4*>(qq + HALF);
-                  float t = acc[gq];
-                  t = fmaf(k0[0], qa.x, t); t = fmaf(k1[0], qb.x, t);
-                  t = fmaf(k0[1], qa.y, t); t = fmaf(k1[1], qb.y, t);
-                  t = fmaf(k0[2], qa.z, t); t = fmaf(k1[2], qb.z, t);
-                  t = fmaf(k0[3], qa.w, t); t = fmaf(k1[3], qb.w, t);
-                  acc[gq] = t;
-                }
+                sc[sl * G + gq] = t;
               }
             }
           }
-#pragma unroll
-          for (int gq = 0; gq < G; ++gq) sc[hs * G + gq] = rv ? acc[gq] : -INFINITY;
         }
+        // (4) release the accumulator
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -537,56 +561,94 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         }
         ab ^= 1;
         if (ab == 0) aph ^= 1u;
-        // (4) tile-local softmax statistics (log2 domain: scores carry log2(e)/sqrt(d))
+        // (5) exchange the partial scores; abort snapshot for both warpgroups
 #pragma unroll
-        for (int hq = 0; hq < QPW; ++hq) {
-          const float m = warp_max(sc[hq]);
-          if (lane == 0) red[hq * 4 + quad] = m;
-        }
-        if (row == 0) s_stop[wg] = *wc.abort_flag;
-        named_bar(1 + wg, 128);
-        if (s_stop[wg]) { stop = true; break; }
-        float mx[QPW];
+        for (int i = 0; i < QPC; ++i) sPart[(wg * QPC + i) * kTile + row] = sc[i];
+        if (et == 0) s_stop[0] = *wc.abort_flag;
+        named_bar(1, 256);
+        if (s_stop[0]) { stop = true; break; }
+        // (6) softmax of the owned heads (log2 domain: scores carry log2(e)/sqrt(d))
+        constexpr int OQ = ((HPC + 1) / 2) * G;  // owned query heads (upper bound)
+        float scr[OQ], mx[OQ], lsum[OQ];
 #pragma unroll
-        for (int hq = 0; hq < QPW; ++hq) {
-          mx[hq] = fmaxf(fmaxf(red[hq * 4 + 0], red[hq * 4 + 1]), fmaxf(red[hq * 4 + 2], red[hq * 4 + 3]));
-          const float pe = rv ? exp2f(sc[hq] - mx[hq]) : 0.f;
-          p_s[hq * kTile + row] = pe;
-          const float s = warp_sum(pe);
-          if (lane == 0) red[QPW * 4 + hq * 4 + quad] = s;
+        for (int oq = 0; oq < OQ; ++oq) {
+          const int hq = own0 * G + oq;
+          const bool ok_h = oq < own_n * G && own0 + oq / G < hpc;
+          scr[oq] = (rv && ok_h) ? sPart[hq * kTile + row] + sPart[(QPC + hq) * kTile + row]
+                                 : -INFINITY;
+          const float m = warp_max(scr[oq]);
+          if (lane == 0) red[oq * 4 + quad] = m;
         }
-        named_bar(1 + wg, 128);
-        // (5) value latents of this chunk
+        named_bar(2 + wg, 128);
+#pragma unroll
+        for (int oq = 0; oq < OQ; ++oq) {
+          mx[oq] = fmaxf(fmaxf(red[oq * 4 + 0], red[oq * 4 + 1]), fmaxf(red[oq * 4 + 2], red[oq * 4 + 3]));
+          const float pe = rv && scr[oq] > -INFINITY ? exp2f(scr[oq] - mx[oq]) : 0.f;
+          // slots beyond this launch's heads per chunk belong to the other warpgroup
+          if (oq < own_n * G && own0 + oq / G < hpc) sP[(own0 * G + oq) * kTile + row] = pe;
+          const float sm = warp_sum(pe);
+          if (lane == 0) red[OQ * 4 + oq * 4 + quad] = sm;
+        }
+        named_bar(2 + wg, 128);
+#pragma unroll
+        for (int oq = 0; oq < OQ; ++oq)
+          lsum[oq] = red[OQ * 4 + oq * 4 + 0] + red[OQ * 4 + oq * 4 + 1] +
+                     red[OQ * 4 + oq * 4 + 2] + red[OQ * 4 + oq * 4 + 3];
+        // (7) value latents of this chunk, then the latent P.C_v of the owned heads: threads
+        // split the 128 tokens into TG groups, one channel each; partials meet in shared memory
         wait_bounded(bar(B_VF + vs), vph, wc);
-        // (6) latent P.C_v and the partial record of each query head
         const uint8_t* vslot0 = sV + (vs * 2) * p.vslot;
         const int vbase = p.vchunk_off[c];
 #pragma unroll
-        for (int hs = 0; hs < HPW; ++hs) {
-          const int g = g_first + hs;
-          if (g >= p.Hkv || hs >= wg_slots || !has_rows) continue;
+        for (int os = 0; os < (HPC + 1) / 2; ++os) {
+          const int sl = own0 + os;
+          const int g = g0 + sl;
+          const bool live = os < own_n && sl < hpc && g < p.Hkv && has_rows;  // WG-uniform
+          if (!live) continue;
           const LatDesc& vd = p.vh[g];
-          if (row < vd.rank) {
-            float a[G];
+          const int r = vd.rank;
+          const int TG = r <= 32 ? 4 : (r <= 64 ? 2 : 1);
+          const int CW = kTile / TG, TL = kTile / TG;
+          const int ch = row % CW, tg = row / CW;
+          float a0[G], a1[G];
 #pragma unroll
-            for (int gq = 0; gq < G; ++gq) a[gq] = 0.f;
+          for (int gq = 0; gq < G; ++gq) a0[gq] = a1[gq] = 0.f;
+          if (ch < r) {
+#pragma unroll
             for (int pp = 0; pp < 2; ++pp) {
               if (U.page(pp) < 0) continue;
               const uint8_t* slot = vslot0 + pp * p.vslot;
-              const int t1 = min(kPage, U.nvalid - pp * kPage);
-#pragma unroll 4
-              for (int t = 0; t < t1; ++t) {
-                const float cv = vload<FMT>(slot, vd, vbase, t, row);
+              const int t0 = max(tg * TL, pp * kPage);
+              const int t1 = min(min((tg + 1) * TL, pp * kPage + kPage), U.nvalid);
+              int t = t0;
+              for (; t + 1 < t1; t += 2) {
+                const float c0 = vload<FMT>(slot, vd, vbase, t - pp * kPage, ch);
+                const float c1 = vload<FMT>(slot, vd, vbase, t + 1 - pp * kPage, ch);
 #pragma unroll
-                for (int gq = 0; gq < G; ++gq)
-                  a[gq] = fmaf(p_s[(hs * G + gq) * kTile + pp * kPage + t], cv, a[gq]);
+                for (int gq = 0; gq < G; ++gq) {
+                  const float* pr = sP + (sl * G + gq) * kTile;
+                  a0[gq] = fmaf(pr[t], c0, a0[gq]);
+                  a1[gq] = fmaf(pr[t + 1], c1, a1[gq]);
+                }
+              }
+              if (t < t1) {
+                const float c0 = vload<FMT>(slot, vd, vbase, t - pp * kPage, ch);
+#pragma unroll
+                for (int gq = 0; gq < G; ++gq) a0[gq] = fmaf(sP[(sl * G + gq) * kTile + t], c0, a0[gq]);
               }
             }
+          }
+#pragma unroll
+          for (int gq = 0; gq < G; ++gq) pv[gq * kTile + row] = a0[gq] + a1[gq];
+          named_bar(2 + wg, 128);
+          if (tg == 0 && ch < r) {
 #pragma unroll
             for (int gq = 0; gq < G; ++gq) {
+              float a = 0.f;
+              for (int k = 0; k < TG; ++k) a += pv[gq * kTile + k * CW + ch];
               const int h = g * G + gq;
               float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
-              rec[2 + row] = a[gq];
+              rec[2 + ch] = a;
             }
           }
           if (row == 0) {
@@ -594,13 +656,13 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             for (int gq = 0; gq < G; ++gq) {
               const int h = g * G + gq;
               float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
-              const int hq = hs * G + gq;
-              rec[0] = mx[hq];
-              rec[1] = red[QPW * 4 + hq * 4 + 0] + red[QPW * 4 + hq * 4 + 1] +
-                       red[QPW * 4 + hq * 4 + 2] + red[QPW * 4 + hq * 4 + 3];
+              rec[0] = mx[os * G + gq];
+              rec[1] = lsum[os * G + gq];
             }
           }
+          named_bar(2 + wg, 128);  // pv is reused by the next owned head
         }
+        // (8) release the value buffer
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_VE + vs));
         if (++vs == NVB) { vs = 0; vph ^= 1u; }
@@ -773,6 +835,14 @@ static cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tmA,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (CG > 1) {
+    // a persistent grid must be co-resident: not every SM can host half of a CTA pair
+    // (pairs stay inside a GPC), so cap the grid at the pairs that fit at once
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (clusters >= 1 && grid > clusters * CG) cfg.gridDim = dim3(clusters * CG, 1, 1);
+  }
   return cudaLaunchKernelEx(&cfg, kern, p, tmA, tmB);
 }
 

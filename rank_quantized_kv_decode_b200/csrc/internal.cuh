@@ -66,7 +66,7 @@ struct DecodeParams {
   float qscale;  // log2(e) / sqrt(d)
   // dynamic shared-memory plan (offsets from the 1024-aligned base)
   int stages, nvb, vslot;
-  uint32_t off_b, off_v, off_q, off_p, off_red, off_ang, off_bar, smem_bytes;
+  uint32_t off_b, off_v, off_q, off_p, off_part, off_red, off_ang, off_pv, off_bar, smem_bytes;
   LatDesc key;
   int vchunk_off[kMaxChunks];
   int vchunk_bytes[kMaxChunks];

@@ -225,12 +225,17 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive (optionally announcing transaction bytes) on an mbarrier of any CTA of the cluster.
+// Arrive on an mbarrier of any CTA of the cluster.  The release is at cluster scope: use it
+// when this thread's earlier writes (shared memory read by the peer's MMAs, TMEM reads that
+// must finish before the peer overwrites) have to be ordered before the arrival.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Announce transaction bytes on an mbarrier of any CTA of the cluster.  Default semantics: the
+// data itself is published by the copies' complete_tx, the arrival orders nothing else, so
+// no cluster-scope fence is paid on the producer's critical path.
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr, uint32_t tx) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_addr),
                "r"(tx)
                : "memory");
 }
@@ -282,6 +287,21 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask
           bar),
       "h"(cta_mask)
       : "memory");
+}
+
+// Asynchronous pair of 32-lane x 8-column TMEM loads (no wait).  The registers are valid only
+// after tmem_wait_regs16 on the same array: that wait names them as in/out operands, so the
+// compiler cannot move their uses above it.
+__device__ __forceinline__ void tmem_ld8x2(uint32_t taddr0, uint32_t taddr1, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%16];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%17];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr0), "r"(taddr1)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_regs16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]) : : "memory");
 }
 
 // Nearest tf32 value (ties away from zero) of an fp32 value, returned as fp32 with the low 13
