@@ -468,26 +468,47 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       const int T = U.L - 1;  // position of the decode query
       const bool rv = row < U.nvalid && U.page(row >> 6) >= 0;
       const bool has_rows = U.nvalid > 0;  // a pair's second half may lie past the end
+      // queries of a chunk are loaded one chunk ahead (QI values per thread at most)
+      constexpr int QI = (QPC * HALF + 255) / 256;
+      float qx0[QI], qx1[QI];
+      auto load_q = [&](int cc) {
+#pragma unroll
+        for (int k = 0; k < QI; ++k) {
+          const int idx = et + 256 * k;
+          const int hq = idx / HALF, j = idx % HALF;
+          const int g = cc * hpc + hq / G;
+          qx0[k] = qx1[k] = 0.f;
+          if (idx < hpc * G * HALF && g < p.Hkv) {
+            const long long qb = ((long long)U.b * p.H + g * G + hq % G) * HD;
+            qx0[k] = qload<FMT>(p.q, qb + j);
+            qx1[k] = qload<FMT>(p.q, qb + j + HALF);
+          }
+        }
+      };
+      load_q(U.c0);
+      // rotation of the query at position T: the same for every head
       for (int c = U.c0; c < U.c1; ++c) {
         const int g0 = c * hpc;  // first KV head of the chunk
         // (1) rotated, scaled queries of every head of the chunk; the tile's start angles
-        for (int idx = et; idx < hpc * G * HALF; idx += 256) {
+#pragma unroll
+        for (int k = 0; k < QI; ++k) {
+          const int idx = et + 256 * k;
           const int hq = idx / HALF, j = idx % HALF;
-          const int g = g0 + hq / G;
-          if (g >= p.Hkv) continue;
-          const int h = g * G + hq % G;
-          const long long qb = ((long long)U.b * p.H + h) * HD;
-          const float x0 = qload<FMT>(p.q, qb + j), x1 = qload<FMT>(p.q, qb + j + HALF);
-          const float2 bs = basetab[(T >> 7) * HALF + j], f = fine[(T & 127) * HALF + j];
-          const float cs = bs.x * f.x - bs.y * f.y, sn = bs.y * f.x + bs.x * f.y;
-          sQ[hq * HD + j] = (x0 * cs - x1 * sn) * p.qscale;
-          sQ[hq * HD + j + HALF] = (x1 * cs + x0 * sn) * p.qscale;
+          if (idx < hpc * G * HALF) {
+            const float2 bs = basetab[(T >> 7) * HALF + j], f = fine[(T & 127) * HALF + j];
+            const float cs = bs.x * f.x - bs.y * f.y, sn = bs.y * f.x + bs.x * f.y;
+            sQ[hq * HD + j] = (qx0[k] * cs - qx1[k] * sn) * p.qscale;
+            sQ[hq * HD + j + HALF] = (qx1[k] * cs + qx0[k] * sn) * p.qscale;
+          }
         }
-        for (int j = et; j < HALF; j += 256) {
-          const float2 bs = basetab[min(U.tile, p.rope_tiles - 1) * HALF + j];
-          phi_s[j] = atan2f(bs.y, bs.x);
+        if (c == U.c0) {
+          for (int j = et; j < HALF; j += 256) {
+            const float2 bs = basetab[min(U.tile, p.rope_tiles - 1) * HALF + j];
+            phi_s[j] = atan2f(bs.y, bs.x);
+          }
         }
         named_bar(1, 256);
+        if (c + 1 < U.c1) load_q(c + 1);  // in flight while the accumulator is computed
         // (2) accumulator of this chunk (on a timeout the data is garbage and the snapshot
         // below ends the loop)
         wait_bounded(bar(B_ACCF + ab), aph, wc);
@@ -535,27 +556,27 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
 #pragma unroll
               for (int gq = 0; gq < G; ++gq) {
                 const float* qq = sQ + (sl * G + gq) * HD + j0;
-                float t = sc[sl * G + gq];
+                float t0 = 0.f, t1 = 0.f;  // two chains
 #pragma unroll
                 for (int e = 0; e < JG; e += 4) {
                   const float4 qa = *reinterpret_cast<const float4*>(qq + e);
                   const float4 qb = *reinterpret_cast<const float4*>(qq + HALF + e);
-                  t = fmaf(k0[e + 0], qa.x, t); t = fmaf(k1[e + 0], qb.x, t);
-                  t = fmaf(k0[e + 1], qa.y, t); t = fmaf(k1[e + 1], qb.y, t);
-                  t = fmaf(k0[e + 2], qa.z, t); t = fmaf(k1[e + 2], qb.z, t);
-                  t = fmaf(k0[e + 3], qa.w, t); t = fmaf(k1[e + 3], qb.w, t);
+                  t0 = fmaf(k0[e + 0], qa.x, t0); t1 = fmaf(k1[e + 0], qb.x, t1);
+                  t0 = fmaf(k0[e + 1], qa.y, t0); t1 = fmaf(k1[e + 1], qb.y, t1);
+                  t0 = fmaf(k0[e + 2], qa.z, t0); t1 = fmaf(k1[e + 2], qb.z, t1);
+                  t0 = fmaf(k0[e + 3], qa.w, t0); t1 = fmaf(k1[e + 3], qb.w, t1);
                 }
-                sc[sl * G + gq] = t;
+                sc[sl * G + gq] += t0 + t1;
               }
             }
           }
         }
-        // (4) release the accumulator
+        // (4) release the accumulator (the loads have completed at their wait::ld)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           if (CG == 2 && !leader)
-            mbar_arrive_cluster(leader_bar(B_ACCE + ab));
+            mbar_arrive_remote(leader_bar(B_ACCE + ab));
           else
             mbar_arrive(bar(B_ACCE + ab));
         }

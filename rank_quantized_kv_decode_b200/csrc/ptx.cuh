@@ -231,6 +231,12 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Arrive on an mbarrier of any CTA of the cluster with default (CTA-scope release) semantics:
+// for arrivals that order nothing a peer reads, e.g. a TMEM buffer release after
+// tcgen05.wait::ld has already completed the loads.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 // Announce transaction bytes on an mbarrier of any CTA of the cluster.  Default semantics: the
 // data itself is published by the copies' complete_tx, the arrival orders nothing else, so
 // no cluster-scope fence is paid on the producer's critical path.
