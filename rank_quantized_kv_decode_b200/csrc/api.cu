@@ -534,6 +534,13 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   }
   for (int g = 0; g < c.n_kv_heads; ++g) p.vh[g] = lat_desc(lay->seg[1 + g]);
 
+  // int8/int4 keys of rank <= 256 keep the dequantised tile resident for all its chunks
+  const bool ares = fmt == STARKV_FMT_MIXED && p.kb_count <= 4;
+  p.a_resident = ares ? 1 : 0;
+  {
+    const starkv_segment& k = lay->seg[0];
+    p.key_region = ares ? static_cast<int>(k.off_sc + int64_t(kPage) * 2 * (k.g8 + k.g4) - k.off_i8) : 0;
+  }
   // shared-memory plan: ring stages of (A k-block, B k-block), value buffers, small arrays
   p.vslot = (vmax + 127) / 128 * 128;
   const size_t bstage = static_cast<size_t>(p.NC / CG) * kKBytes;
@@ -544,9 +551,11 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     size_t off = 0;
     const int S = pl[0], NVB = pl[1];
     const size_t split = fmt == STARKV_FMT_F32 ? 2 : 1;  // hi/lo copies for 3xTF32
-    off += S * split * static_cast<size_t>(kAStage);
+    off += (ares ? p.kb_count : S) * split * static_cast<size_t>(kAStage);
     const size_t off_b = off;
     off += S * split * bstage;
+    const size_t off_codes = off;
+    off += ares ? 2 * 2 * static_cast<size_t>(p.key_region) : 0;
     const size_t off_v = off;
     off += static_cast<size_t>(NVB) * 2 * p.vslot;
     const size_t QPC = static_cast<size_t>(256 / d) * p.G;  // query heads of a full chunk
@@ -565,7 +574,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     off += 2 * static_cast<size_t>(p.G) * kTile * 4;
     off = (off + 7) / 8 * 8;
     const size_t off_bar = off;
-    off += (3 * S + 4 + 2 * NVB + 1) * 8 + 16;
+    off += (3 * S + 4 + 2 * NVB + 1 + 12) * 8 + 16;
     // alignment slack of the dynamic base; at least 120 KB so that one CTA occupies an SM
     // (each CTA allocates all 512 TMEM columns)
     const size_t total = std::max<size_t>(off + 1024, 120 * 1024);
@@ -573,6 +582,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
       p.stages = S;
       p.nvb = NVB;
       p.off_b = static_cast<uint32_t>(off_b);
+      p.off_codes = static_cast<uint32_t>(off_codes);
       p.off_v = static_cast<uint32_t>(off_v);
       p.off_q = static_cast<uint32_t>(off_q);
       p.off_p = static_cast<uint32_t>(off_p);

@@ -118,6 +118,73 @@ __device__ __forceinline__ float vload(const uint8_t* slot, const LatDesc& vd, i
   }
 }
 
+// One value-latent channel of one KV head in a staged page slot, with everything that does
+// not depend on the token hoisted: byte offset and token stride of its code (or value), and
+// for int8/int4 its scale's offset/stride, the nibble shift and whether it is an int8 channel.
+struct VChan {
+  int off, stride;
+  int soff, sstride;
+  int shift;
+  bool is8;
+};
+
+template <int FMT>
+__device__ __forceinline__ VChan vchan(const LatDesc& vd, int vbase, int i) {
+  VChan v{};
+  if constexpr (FMT == FMT_F32) {
+    v.off = vd.off0 - vbase + 4 * i;
+    v.stride = 4 * vd.rank;
+  } else if constexpr (FMT == FMT_BF16) {
+    v.off = vd.off0 - vbase + 2 * i;
+    v.stride = 2 * vd.rank;
+  } else {
+    v.is8 = i < vd.n8;
+    const int j = i - vd.n8;
+    v.off = v.is8 ? vd.off0 - vbase + i : vd.off1 - vbase + (j >> 1);
+    v.stride = v.is8 ? vd.n8 : vd.nb4;
+    v.shift = v.is8 ? 0 : (j & 1) * 4;
+    v.soff = vd.off2 - vbase + 2 * (v.is8 ? (i >> 5) : vd.g8 + (j >> 5));
+    v.sstride = 2 * vd.ng;
+  }
+  return v;
+}
+
+template <int FMT>
+__device__ __forceinline__ float vchan_load(const uint8_t* slot, const VChan& v, int row) {
+  if constexpr (FMT == FMT_F32) {
+    return *reinterpret_cast<const float*>(slot + v.off + row * v.stride);
+  } else if constexpr (FMT == FMT_BF16) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(slot + v.off + row * v.stride));
+  } else {
+    const int b = slot[v.off + row * v.stride];
+    const int q = v.is8 ? static_cast<int>(static_cast<int8_t>(b)) : (((b >> v.shift) & 15) ^ 8) - 8;
+    const float s = __half2float(*reinterpret_cast<const __half*>(slot + v.soff + row * v.sstride));
+    return s * static_cast<float>(q);
+  }
+}
+
+// The G probabilities of one token for one GQA group (contiguous in the token-major layout).
+template <int G>
+__device__ __forceinline__ void load_p(const float* ptr, float (&out)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int k = 0; k < G; k += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(ptr + k);
+      out[k] = v.x;
+      out[k + 1] = v.y;
+      out[k + 2] = v.z;
+      out[k + 3] = v.w;
+    }
+  } else if constexpr (G == 2) {
+    const float2 v = *reinterpret_cast<const float2*>(ptr);
+    out[0] = v.x;
+    out[1] = v.y;
+  } else {
+#pragma unroll
+    for (int k = 0; k < G; ++k) out[k] = ptr[k];
+  }
+}
+
 // 8 consecutive key-latent channels [k0, k0+8) of one token as fp16 (scale * code, rounded
 // to nearest), packed for one 16-byte store.  ``base`` is the page.
 __device__ __forceinline__ float key_code_value(const uint8_t* base, const LatDesc& kd, int prow,
@@ -138,13 +205,12 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ uint4 dequant8(const DecodeParams& p, const Unit& U, int r, int k0) {
+// Channels [k0, k0+8) of token row ``prow`` of a page whose key blocks are at ``base`` + the
+// offsets of ``kd`` (the page itself in global memory, or a copy of its key region in shared
+// memory with the offsets rebased).
+__device__ __forceinline__ uint4 dequant8_at(const uint8_t* base, const LatDesc& kd, int prow, int k0) {
   uint4 z = make_uint4(0, 0, 0, 0);
-  const int pp = r >> 6, prow = r & 63;
-  const int pg = U.page(pp);
-  const LatDesc& kd = p.key;
-  if (pg < 0 || r >= U.nvalid || k0 >= kd.rank) return z;
-  const uint8_t* base = p.cache + (long long)pg * p.page_bytes;
+  if (k0 >= kd.rank) return z;
   float v[8];
   if (k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0) {
     const uint2 raw = *reinterpret_cast<const uint2*>(base + kd.off0 + prow * kd.n8 + k0);
@@ -176,6 +242,14 @@ __device__ __forceinline__ uint4 dequant8(const DecodeParams& p, const Unit& U, 
   z.z = pack_h2(v[4], v[5]);
   z.w = pack_h2(v[6], v[7]);
   return z;
+}
+
+// Row r of the tile's operand, read from the pages in global memory.
+__device__ __forceinline__ uint4 dequant8(const DecodeParams& p, const Unit& U, int r, int k0) {
+  const int pp = r >> 6, prow = r & 63;
+  const int pg = U.page(pp);
+  if (pg < 0 || r >= U.nvalid) return make_uint4(0, 0, 0, 0);
+  return dequant8_at(p.cache + (long long)pg * p.page_bytes, p.key, prow, k0);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -234,17 +308,32 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   const int B_FULL = 0, B_EMPTY = S, B_RAW = 2 * S, B_ACCF = 3 * S, B_ACCE = 3 * S + 2,
             B_VF = 3 * S + 4, B_VE = 3 * S + 4 + NVB, B_TD = 3 * S + 4 + 2 * NVB;
+  // resident operand (int8/int4 keys of rank <= 256): dequantised once per tile into kb_count
+  // slots, each used by every chunk of the unit; the tile's codes are staged by bulk copy
+  const int B_AF = B_TD + 1, B_AE = B_AF + 4, B_CF = B_AE + 4, B_CE = B_CF + 2;
+  const bool ares = !F::kTmaA && p.a_resident;
+  uint8_t* sCodes = smem + p.off_codes;  // [2 buffers][2 pages][key_region]
   // misc: [0] TMEM base, [1] abort flag, [2..3] per-warpgroup stop snapshots
-  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + B_TD + 1);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + B_CE + 2);
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   if (threadIdx.x == 0) {
     // a pair's full barriers (in the leader) count both CTAs' producers and dequantisers;
     // its accumulator-empty barriers count the epilogue warps of both CTAs
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar(B_FULL + s), CG == 1 ? F::kFullCount : (F::kTmaA ? 2 : 10));
+      // the resident operand is not part of a ring stage: only the producers arrive
+      const int full = ares ? CG : (CG == 1 ? F::kFullCount : (F::kTmaA ? 2 : 10));
+      mbar_init(bar(B_FULL + s), full);
       mbar_init(bar(B_EMPTY + s), 1);
       mbar_init(bar(B_RAW + s), 1);
+    }
+    for (int k = 0; k < 4; ++k) {
+      mbar_init(bar(B_AF + k), 4 * CG);
+      mbar_init(bar(B_AE + k), 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(bar(B_CF + k), 1);
+      mbar_init(bar(B_CE + k), 4);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(B_ACCF + a), 1);
@@ -345,19 +434,22 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && leader) {
       int stage = 0, ab = 0;
-      uint32_t phase = 0, aph = 0;
+      uint32_t phase = 0, aph = 0, uc = 0;
       bool ok = true;
       for (int u = unit0; ok && u < p.total_units; u += unit_step) {
         Unit U;
         if (!get_unit<CG>(p, u, U, false, crank)) continue;
+        ++uc;
         for (int c = U.c0; ok && c < U.c1; ++c) {
           if (!wait_bounded(bar(B_ACCE + ab), aph ^ 1u, wc)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * 256);
           for (int kb = 0; kb < p.kb_count; ++kb) {
+            if (ares && c == U.c0 &&
+                !wait_bounded(bar(B_AF + kb), (uc - 1) & 1u, wc)) { ok = false; break; }
             if (!wait_bounded(bar(B_FULL + stage), phase, wc)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t da = desc_sw128(smem_u32(sA + stage * astride));
+            const uint64_t da = desc_sw128(smem_u32(sA + (ares ? kb : stage) * astride));
             const uint64_t db = desc_sw128(smem_u32(sB + stage * bstride));
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -373,11 +465,15 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
                 }
               }
             }
-            // the stage is free in both CTAs once these MMAs have read it
-            if constexpr (CG == 2)
+            // the stage is free in both CTAs once these MMAs have read it; a resident slot
+            // once the unit's last chunk has
+            if constexpr (CG == 2) {
               umma_commit_pair(bar(B_EMPTY + stage), 3);
-            else
+              if (ares && c + 1 == U.c1) umma_commit_pair(bar(B_AE + kb), 3);
+            } else {
               umma_commit(bar(B_EMPTY + stage));
+              if (ares && c + 1 == U.c1) umma_commit(bar(B_AE + kb));
+            }
             if (++stage == S) { stage = 0; phase ^= 1u; }
           }
           if (!ok) break;
@@ -423,6 +519,31 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       }
       for (int v = 0; v < NVB; ++v)
         if (issued & (1u << v)) wait_drain(bar(B_VF + v), (last_phase >> v) & 1u, p.timeout_ns);
+    }
+  } else if (warp == 3) {
+    // ---------------------------------------------------------------- key-code stager
+    if (ares && lane == 0) {
+      const uint32_t kreg = static_cast<uint32_t>(p.key_region);
+      int cb = 0;
+      uint32_t cph = 0, issued = 0, last_phase = 0;
+      for (int u = unit0; u < p.total_units; u += unit_step) {
+        Unit U;
+        if (!get_unit<CG>(p, u, U, false, crank)) continue;
+        if (!wait_bounded(bar(B_CE + cb), cph ^ 1u, wc)) break;
+        const uint32_t fb = bar(B_CF + cb);
+        mbar_arrive_expect_tx(fb, kreg * ((U.page0 >= 0) + (U.page1 >= 0)));
+        for (int pp = 0; pp < 2; ++pp) {
+          const int pg = U.page(pp);
+          if (pg < 0) continue;
+          bulk_g2s(smem_u32(sCodes + (cb * 2 + pp) * kreg),
+                   p.cache + (long long)pg * p.page_bytes + p.key.off0, kreg, fb);
+        }
+        issued |= 1u << cb;
+        last_phase = (last_phase & ~(1u << cb)) | (cph << cb);
+        if (++cb == 2) { cb = 0; cph ^= 1u; }
+      }
+      for (int k = 0; k < 2; ++k)
+        if (issued & (1u << k)) wait_drain(bar(B_CF + k), (last_phase >> k) & 1u, p.timeout_ns);
     }
   } else if (warp >= 4 && warp < 12) {
     // ---------------------------------------------------------------- epilogue warpgroups
@@ -588,9 +709,10 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         if (et == 0) s_stop[0] = *wc.abort_flag;
         named_bar(1, 256);
         if (s_stop[0]) { stop = true; break; }
-        // (6) softmax of the owned heads (log2 domain: scores carry log2(e)/sqrt(d))
+        // (6) softmax of the owned heads (log2 domain: scores carry log2(e)/sqrt(d));
+        // probabilities stored token-major, [row][QPC], so one vector load serves a GQA group
         constexpr int OQ = ((HPC + 1) / 2) * G;  // owned query heads (upper bound)
-        float scr[OQ], mx[OQ], lsum[OQ];
+        float scr[OQ];
 #pragma unroll
         for (int oq = 0; oq < OQ; ++oq) {
           const int hq = own0 * G + oq;
@@ -603,18 +725,15 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         named_bar(2 + wg, 128);
 #pragma unroll
         for (int oq = 0; oq < OQ; ++oq) {
-          mx[oq] = fmaxf(fmaxf(red[oq * 4 + 0], red[oq * 4 + 1]), fmaxf(red[oq * 4 + 2], red[oq * 4 + 3]));
-          const float pe = rv && scr[oq] > -INFINITY ? exp2f(scr[oq] - mx[oq]) : 0.f;
+          const float mxv = fmaxf(fmaxf(red[oq * 4 + 0], red[oq * 4 + 1]),
+                                  fmaxf(red[oq * 4 + 2], red[oq * 4 + 3]));
+          const float pe = rv && scr[oq] > -INFINITY ? exp2f(scr[oq] - mxv) : 0.f;
           // slots beyond this launch's heads per chunk belong to the other warpgroup
-          if (oq < own_n * G && own0 + oq / G < hpc) sP[(own0 * G + oq) * kTile + row] = pe;
+          if (oq < own_n * G && own0 + oq / G < hpc) sP[row * QPC + own0 * G + oq] = pe;
           const float sm = warp_sum(pe);
           if (lane == 0) red[OQ * 4 + oq * 4 + quad] = sm;
         }
         named_bar(2 + wg, 128);
-#pragma unroll
-        for (int oq = 0; oq < OQ; ++oq)
-          lsum[oq] = red[OQ * 4 + oq * 4 + 0] + red[OQ * 4 + oq * 4 + 1] +
-                     red[OQ * 4 + oq * 4 + 2] + red[OQ * 4 + oq * 4 + 3];
         // (7) value latents of this chunk, then the latent P.C_v of the owned heads: threads
         // split the 128 tokens into TG groups, one channel each; partials meet in shared memory
         wait_bounded(bar(B_VF + vs), vph, wc);
@@ -631,9 +750,10 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           const int TG = r <= 32 ? 4 : (r <= 64 ? 2 : 1);
           const int CW = kTile / TG, TL = kTile / TG;
           const int ch = row % CW, tg = row / CW;
-          float a0[G], a1[G];
+          const VChan vc = vchan<FMT>(vd, vbase, ch);
+          float a[G];
 #pragma unroll
-          for (int gq = 0; gq < G; ++gq) a0[gq] = a1[gq] = 0.f;
+          for (int gq = 0; gq < G; ++gq) a[gq] = 0.f;
           if (ch < r) {
 #pragma unroll
             for (int pp = 0; pp < 2; ++pp) {
@@ -641,44 +761,38 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
               const uint8_t* slot = vslot0 + pp * p.vslot;
               const int t0 = max(tg * TL, pp * kPage);
               const int t1 = min(min((tg + 1) * TL, pp * kPage + kPage), U.nvalid);
-              int t = t0;
-              for (; t + 1 < t1; t += 2) {
-                const float c0 = vload<FMT>(slot, vd, vbase, t - pp * kPage, ch);
-                const float c1 = vload<FMT>(slot, vd, vbase, t + 1 - pp * kPage, ch);
+#pragma unroll 4
+              for (int t = t0; t < t1; ++t) {
+                const float cv = vchan_load<FMT>(slot, vc, t - pp * kPage);
+                float pr[G];
+                load_p<G>(sP + t * QPC + sl * G, pr);
 #pragma unroll
-                for (int gq = 0; gq < G; ++gq) {
-                  const float* pr = sP + (sl * G + gq) * kTile;
-                  a0[gq] = fmaf(pr[t], c0, a0[gq]);
-                  a1[gq] = fmaf(pr[t + 1], c1, a1[gq]);
-                }
-              }
-              if (t < t1) {
-                const float c0 = vload<FMT>(slot, vd, vbase, t - pp * kPage, ch);
-#pragma unroll
-                for (int gq = 0; gq < G; ++gq) a0[gq] = fmaf(sP[(sl * G + gq) * kTile + t], c0, a0[gq]);
+                for (int gq = 0; gq < G; ++gq) a[gq] = fmaf(pr[gq], cv, a[gq]);
               }
             }
           }
 #pragma unroll
-          for (int gq = 0; gq < G; ++gq) pv[gq * kTile + row] = a0[gq] + a1[gq];
+          for (int gq = 0; gq < G; ++gq) pv[gq * kTile + row] = a[gq];
           named_bar(2 + wg, 128);
           if (tg == 0 && ch < r) {
 #pragma unroll
             for (int gq = 0; gq < G; ++gq) {
-              float a = 0.f;
-              for (int k = 0; k < TG; ++k) a += pv[gq * kTile + k * CW + ch];
+              float acc = 0.f;
+              for (int k = 0; k < TG; ++k) acc += pv[gq * kTile + k * CW + ch];
               const int h = g * G + gq;
               float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
-              rec[2 + ch] = a;
+              rec[2 + ch] = acc;
             }
           }
           if (row == 0) {
 #pragma unroll
             for (int gq = 0; gq < G; ++gq) {
+              const int oq = os * G + gq;
               const int h = g * G + gq;
               float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
-              rec[0] = mx[os * G + gq];
-              rec[1] = lsum[os * G + gq];
+              rec[0] = fmaxf(fmaxf(red[oq * 4 + 0], red[oq * 4 + 1]), fmaxf(red[oq * 4 + 2], red[oq * 4 + 3]));
+              rec[1] = red[OQ * 4 + oq * 4 + 0] + red[OQ * 4 + oq * 4 + 1] +
+                       red[OQ * 4 + oq * 4 + 2] + red[OQ * 4 + oq * 4 + 3];
             }
           }
           named_bar(2 + wg, 128);  // pv is reused by the next owned head
@@ -720,7 +834,51 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       }
     }
     // ---------------------------------------------------------------- dequantisers (int8/int4)
-    if constexpr (!F::kTmaA) {
+    if (!F::kTmaA && ares) {
+      // once per tile, from the staged codes, into the resident slots
+      const int tid = (warp - 12) * 32 + lane;
+      const int ch = tid & 7;
+      LatDesc kd = p.key;  // offsets rebased onto the staged key region
+      kd.off1 -= kd.off0;
+      kd.off2 -= kd.off0;
+      kd.off0 = 0;
+      const int kreg = p.key_region;
+      int cb = 0;
+      uint32_t cph = 0, uc = 0;
+      bool ok = true;
+      for (int u = unit0; ok && u < p.total_units; u += unit_step) {
+        Unit U;
+        if (!get_unit<CG>(p, u, U, false, crank)) continue;
+        if (!__all_sync(0xffffffffu, wait_bounded(bar(B_CF + cb), cph, wc))) break;
+        for (int kb = 0; kb < p.kb_count; ++kb) {
+          if (!__all_sync(0xffffffffu, wait_bounded(bar(B_AE + kb), (uc & 1u) ^ 1u, wc))) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = sA + kb * kAStage;
+#pragma unroll 2
+          for (int it = 0; it < 8; ++it) {
+            const int r = it * 16 + (tid >> 3);
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r < U.nvalid && U.page(r >> 6) >= 0)
+              v = dequant8_at(sCodes + (cb * 2 + (r >> 6)) * kreg, kd, r & 63, kb * 64 + ch * 8);
+            *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch)) = v;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (CG == 2)
+              mbar_arrive_cluster(leader_bar(B_AF + kb));
+            else
+              mbar_arrive(bar(B_AF + kb));
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_CE + cb));
+        ++uc;
+        if (++cb == 2) { cb = 0; cph ^= 1u; }
+      }
+    } else if constexpr (!F::kTmaA) {
       const int tid = (warp - 12) * 32 + lane;
       int stage = 0;
       uint32_t phase = 0;

@@ -62,11 +62,13 @@ struct DecodeParams {
   int H, Hkv, G, d, rk, key_rank_cols;
   int NC, n_chunks, n_ranges, cpr, kb_count, total_units;
   int cta_group;  // 1: one CTA per 128-token tile; 2: a CTA pair per 256-token tile
+  int a_resident;  // int8/int4 keys: operand dequantised once per tile (kb_count <= 4)
+  int key_region;  // bytes of the key blocks of one page (int8 | int4 | scales)
   uint32_t idesc;
   float qscale;  // log2(e) / sqrt(d)
   // dynamic shared-memory plan (offsets from the 1024-aligned base)
   int stages, nvb, vslot;
-  uint32_t off_b, off_v, off_q, off_p, off_part, off_red, off_ang, off_pv, off_bar, smem_bytes;
+  uint32_t off_b, off_codes, off_v, off_q, off_p, off_part, off_red, off_ang, off_pv, off_bar, smem_bytes;
   LatDesc key;
   int vchunk_off[kMaxChunks];
   int vchunk_bytes[kMaxChunks];
