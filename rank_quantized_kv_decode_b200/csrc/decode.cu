@@ -96,36 +96,13 @@ struct Fmt {
   static constexpr int kFullCount = kSplit ? 4 : (kTmaA ? 1 : 5);
 };
 
-// Stored value of value-latent channel i of token row ``row`` (0..63) in a staged page slot.
-template <int FMT>
-__device__ __forceinline__ float vload(const uint8_t* slot, const LatDesc& vd, int vbase, int row,
-                                       int i) {
-  if constexpr (FMT == FMT_F32) {
-    return reinterpret_cast<const float*>(slot + vd.off0 - vbase)[row * vd.rank + i];
-  } else if constexpr (FMT == FMT_BF16) {
-    return __bfloat162float(
-        reinterpret_cast<const __nv_bfloat16*>(slot + vd.off0 - vbase)[row * vd.rank + i]);
-  } else {
-    const __half* sc = reinterpret_cast<const __half*>(slot + vd.off2 - vbase) + row * vd.ng;
-    if (i < vd.n8) {
-      const int8_t q = reinterpret_cast<const int8_t*>(slot + vd.off0 - vbase)[row * vd.n8 + i];
-      return __half2float(sc[i >> 5]) * static_cast<float>(q);
-    }
-    const int j = i - vd.n8;
-    const uint8_t byte = (slot + vd.off1 - vbase)[row * vd.nb4 + (j >> 1)];
-    const int nib = (j & 1) ? (byte >> 4) : (byte & 15);
-    return __half2float(sc[vd.g8 + (j >> 5)]) * static_cast<float>((nib ^ 8) - 8);
-  }
-}
-
 // One value-latent channel of one KV head in a staged page slot, with everything that does
 // not depend on the token hoisted: byte offset and token stride of its code (or value), and
 // for int8/int4 its scale's offset/stride, the nibble shift and whether it is an int8 channel.
 struct VChan {
   int off, stride;
   int soff, sstride;
-  int shift;
-  bool is8;
+  int lsh, rsh;  // signed code = (byte << lsh) >> rsh: int8 (24, 24), low / high nibble (28 / 24, 28)
 };
 
 template <int FMT>
@@ -138,12 +115,13 @@ __device__ __forceinline__ VChan vchan(const LatDesc& vd, int vbase, int i) {
     v.off = vd.off0 - vbase + 2 * i;
     v.stride = 2 * vd.rank;
   } else {
-    v.is8 = i < vd.n8;
+    const bool is8 = i < vd.n8;
     const int j = i - vd.n8;
-    v.off = v.is8 ? vd.off0 - vbase + i : vd.off1 - vbase + (j >> 1);
-    v.stride = v.is8 ? vd.n8 : vd.nb4;
-    v.shift = v.is8 ? 0 : (j & 1) * 4;
-    v.soff = vd.off2 - vbase + 2 * (v.is8 ? (i >> 5) : vd.g8 + (j >> 5));
+    v.off = is8 ? vd.off0 - vbase + i : vd.off1 - vbase + (j >> 1);
+    v.stride = is8 ? vd.n8 : vd.nb4;
+    v.lsh = is8 ? 24 : ((j & 1) ? 24 : 28);
+    v.rsh = is8 ? 24 : 28;
+    v.soff = vd.off2 - vbase + 2 * (is8 ? (i >> 5) : vd.g8 + (j >> 5));
     v.sstride = 2 * vd.ng;
   }
   return v;
@@ -156,8 +134,8 @@ __device__ __forceinline__ float vchan_load(const uint8_t* slot, const VChan& v,
   } else if constexpr (FMT == FMT_BF16) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(slot + v.off + row * v.stride));
   } else {
-    const int b = slot[v.off + row * v.stride];
-    const int q = v.is8 ? static_cast<int>(static_cast<int8_t>(b)) : (((b >> v.shift) & 15) ^ 8) - 8;
+    const unsigned b = slot[v.off + row * v.stride];
+    const int q = static_cast<int>(b << v.lsh) >> v.rsh;
     const float s = __half2float(*reinterpret_cast<const __half*>(slot + v.soff + row * v.sstride));
     return s * static_cast<float>(q);
   }
@@ -252,17 +230,6 @@ __device__ __forceinline__ uint4 dequant8(const DecodeParams& p, const Unit& U, 
   return dequant8_at(p.cache + (long long)pg * p.page_bytes, p.key, prow, k0);
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 template <int FMT>
 __device__ __forceinline__ float qload(const void* q, long long idx) {
   if constexpr (FMT == FMT_F32) return reinterpret_cast<const float*>(q)[idx];
@@ -271,7 +238,7 @@ __device__ __forceinline__ float qload(const void* q, long long idx) {
 
 }  // namespace
 
-template <int FMT, int HD, int G, int CG>
+template <int FMT, int HD, int G, int CG, int RES>
 __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams p,
                         const __grid_constant__ CUtensorMap tmA,
@@ -311,7 +278,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   // resident operand (int8/int4 keys of rank <= 256): dequantised once per tile into kb_count
   // slots, each used by every chunk of the unit; the tile's codes are staged by bulk copy
   const int B_AF = B_TD + 1, B_AE = B_AF + 4, B_CF = B_AE + 4, B_CE = B_CF + 2;
-  const bool ares = !F::kTmaA && p.a_resident;
+  constexpr bool ares = RES != 0;  // resident operand (int8/int4 keys of rank <= 256)
   uint8_t* sCodes = smem + p.off_codes;  // [2 buffers][2 pages][key_region]
   // misc: [0] TMEM base, [1] abort flag, [2..3] per-warpgroup stop snapshots
   uint32_t* misc = reinterpret_cast<uint32_t*>(bars + B_CE + 2);
@@ -607,7 +574,15 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         }
       };
       load_q(U.c0);
-      // rotation of the query at position T: the same for every head
+      // rotation of the query at position T: the same for every head and chunk (a thread's
+      // pair index et % HALF does not depend on k, 256 being a multiple of HALF)
+      float qcs, qsn;
+      {
+        const int j = et % HALF;
+        const float2 bs = basetab[(T >> 7) * HALF + j], f = fine[(T & 127) * HALF + j];
+        qcs = (bs.x * f.x - bs.y * f.y) * p.qscale;
+        qsn = (bs.y * f.x + bs.x * f.y) * p.qscale;
+      }
       for (int c = U.c0; c < U.c1; ++c) {
         const int g0 = c * hpc;  // first KV head of the chunk
         // (1) rotated, scaled queries of every head of the chunk; the tile's start angles
@@ -616,10 +591,8 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           const int idx = et + 256 * k;
           const int hq = idx / HALF, j = idx % HALF;
           if (idx < hpc * G * HALF) {
-            const float2 bs = basetab[(T >> 7) * HALF + j], f = fine[(T & 127) * HALF + j];
-            const float cs = bs.x * f.x - bs.y * f.y, sn = bs.y * f.x + bs.x * f.y;
-            sQ[hq * HD + j] = (qx0[k] * cs - qx1[k] * sn) * p.qscale;
-            sQ[hq * HD + j + HALF] = (qx1[k] * cs + qx0[k] * sn) * p.qscale;
+            sQ[hq * HD + j] = qx0[k] * qcs - qx1[k] * qsn;
+            sQ[hq * HD + j + HALF] = qx1[k] * qcs + qx0[k] * qsn;
           }
         }
         if (c == U.c0) {
@@ -666,28 +639,36 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
               }
             }
             if (sl < hpc) {
-              float k0[JG], k1[JG];
+              // rotated key pairs, two RoPE pairs per packed register pair:
+              // k0 = a cos - b sin, k1 = b cos + a sin
+              float2 k0[JG / 2], k1[JG / 2];
 #pragma unroll
-              for (int e = 0; e < JG; ++e) {
-                const float a = __uint_as_float(kb[st & 1][e]);
-                const float b = __uint_as_float(kb[st & 1][JG + e]);
-                k0[e] = a * cs[e] - b * sn[e];
-                k1[e] = b * cs[e] + a * sn[e];
+              for (int e = 0; e < JG; e += 2) {
+                const float2 a = make_float2(__uint_as_float(kb[st & 1][e]),
+                                             __uint_as_float(kb[st & 1][e + 1]));
+                const float2 b = make_float2(__uint_as_float(kb[st & 1][JG + e]),
+                                             __uint_as_float(kb[st & 1][JG + e + 1]));
+                const float2 c2 = make_float2(cs[e], cs[e + 1]);
+                const float2 s2 = make_float2(sn[e], sn[e + 1]);
+                const float2 ns2 = make_float2(-sn[e], -sn[e + 1]);
+                k0[e / 2] = __ffma2_rn(b, ns2, __fmul2_rn(a, c2));
+                k1[e / 2] = __ffma2_rn(a, s2, __fmul2_rn(b, c2));
               }
 #pragma unroll
               for (int gq = 0; gq < G; ++gq) {
                 const float* qq = sQ + (sl * G + gq) * HD + j0;
-                float t0 = 0.f, t1 = 0.f;  // two chains
+                float2 t0 = make_float2(0.f, 0.f), t1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int e = 0; e < JG; e += 4) {
                   const float4 qa = *reinterpret_cast<const float4*>(qq + e);
                   const float4 qb = *reinterpret_cast<const float4*>(qq + HALF + e);
-                  t0 = fmaf(k0[e + 0], qa.x, t0); t1 = fmaf(k1[e + 0], qb.x, t1);
-                  t0 = fmaf(k0[e + 1], qa.y, t0); t1 = fmaf(k1[e + 1], qb.y, t1);
-                  t0 = fmaf(k0[e + 2], qa.z, t0); t1 = fmaf(k1[e + 2], qb.z, t1);
-                  t0 = fmaf(k0[e + 3], qa.w, t0); t1 = fmaf(k1[e + 3], qb.w, t1);
+                  t0 = __ffma2_rn(k0[e / 2], make_float2(qa.x, qa.y), t0);
+                  t1 = __ffma2_rn(k1[e / 2], make_float2(qb.x, qb.y), t1);
+                  t0 = __ffma2_rn(k0[e / 2 + 1], make_float2(qa.z, qa.w), t0);
+                  t1 = __ffma2_rn(k1[e / 2 + 1], make_float2(qb.z, qb.w), t1);
                 }
-                sc[sl * G + gq] += t0 + t1;
+                const float2 t = __fadd2_rn(t0, t1);
+                sc[sl * G + gq] += t.x + t.y;
               }
             }
           }
@@ -712,15 +693,24 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         // (6) softmax of the owned heads (log2 domain: scores carry log2(e)/sqrt(d));
         // probabilities stored token-major, [row][QPC], so one vector load serves a GQA group
         constexpr int OQ = ((HPC + 1) / 2) * G;  // owned query heads (upper bound)
-        float scr[OQ];
+        float scr[OQ], rx[OQ];
 #pragma unroll
         for (int oq = 0; oq < OQ; ++oq) {
           const int hq = own0 * G + oq;
           const bool ok_h = oq < own_n * G && own0 + oq / G < hpc;
           scr[oq] = (rv && ok_h) ? sPart[hq * kTile + row] + sPart[(QPC + hq) * kTile + row]
                                  : -INFINITY;
-          const float m = warp_max(scr[oq]);
-          if (lane == 0) red[oq * 4 + quad] = m;
+          rx[oq] = scr[oq];
+        }
+        // warp maxima of all owned heads, the shuffles of different heads interleaved
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+          for (int oq = 0; oq < OQ; ++oq) rx[oq] = fmaxf(rx[oq], __shfl_xor_sync(0xffffffffu, rx[oq], o));
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int oq = 0; oq < OQ; ++oq) red[oq * 4 + quad] = rx[oq];
         }
         named_bar(2 + wg, 128);
 #pragma unroll
@@ -730,12 +720,21 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           const float pe = rv && scr[oq] > -INFINITY ? exp2f(scr[oq] - mxv) : 0.f;
           // slots beyond this launch's heads per chunk belong to the other warpgroup
           if (oq < own_n * G && own0 + oq / G < hpc) sP[row * QPC + own0 * G + oq] = pe;
-          const float sm = warp_sum(pe);
-          if (lane == 0) red[OQ * 4 + oq * 4 + quad] = sm;
+          rx[oq] = pe;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+          for (int oq = 0; oq < OQ; ++oq) rx[oq] += __shfl_xor_sync(0xffffffffu, rx[oq], o);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int oq = 0; oq < OQ; ++oq) red[OQ * 4 + oq * 4 + quad] = rx[oq];
         }
         named_bar(2 + wg, 128);
-        // (7) value latents of this chunk, then the latent P.C_v of the owned heads: threads
-        // split the 128 tokens into TG groups, one channel each; partials meet in shared memory
+        // (7) value latents of this chunk, then the latent P.C_v of the owned heads: thread
+        // row = (token group tg, channel ch) with TG = 128 / r groups of consecutive tokens;
+        // the TG partials of a channel meet in shared memory
         wait_bounded(bar(B_VF + vs), vph, wc);
         const uint8_t* vslot0 = sV + (vs * 2) * p.vslot;
         const int vbase = p.vchunk_off[c];
@@ -746,43 +745,58 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           const bool live = os < own_n && sl < hpc && g < p.Hkv && has_rows;  // WG-uniform
           if (!live) continue;
           const LatDesc& vd = p.vh[g];
-          const int r = vd.rank;
-          const int TG = r <= 32 ? 4 : (r <= 64 ? 2 : 1);
-          const int CW = kTile / TG, TL = kTile / TG;
-          const int ch = row % CW, tg = row / CW;
+          const int r = max(vd.rank, 1);
+          const int TG = kTile / min(r, kTile);
+          const int ch = row % r, tg = row / r;
+          const bool act = tg < TG && ch < vd.rank;
           const VChan vc = vchan<FMT>(vd, vbase, ch);
-          float a[G];
+          constexpr int G2 = (G + 1) / 2;
+          float2 a2[G2];
 #pragma unroll
-          for (int gq = 0; gq < G; ++gq) a[gq] = 0.f;
-          if (ch < r) {
+          for (int k = 0; k < G2; ++k) a2[k] = make_float2(0.f, 0.f);
+          if (act) {
+            const int tlo = (tg * kTile) / TG, thi = ((tg + 1) * kTile) / TG;
 #pragma unroll
             for (int pp = 0; pp < 2; ++pp) {
               if (U.page(pp) < 0) continue;
               const uint8_t* slot = vslot0 + pp * p.vslot;
-              const int t0 = max(tg * TL, pp * kPage);
-              const int t1 = min(min((tg + 1) * TL, pp * kPage + kPage), U.nvalid);
+              const int t0 = max(tlo, pp * kPage);
+              const int t1 = min(min(thi, pp * kPage + kPage), U.nvalid);
 #pragma unroll 4
               for (int t = t0; t < t1; ++t) {
                 const float cv = vchan_load<FMT>(slot, vc, t - pp * kPage);
-                float pr[G];
-                load_p<G>(sP + t * QPC + sl * G, pr);
+                const float* pt = sP + t * QPC + sl * G;
+                if constexpr (G == 1) {
+                  a2[0].x = fmaf(pt[0], cv, a2[0].x);
+                } else {
+                  const float2 cv2 = make_float2(cv, cv);
+                  float pr[G];
+                  load_p<G>(pt, pr);
 #pragma unroll
-                for (int gq = 0; gq < G; ++gq) a[gq] = fmaf(pr[gq], cv, a[gq]);
+                  for (int k = 0; k < G2; ++k)
+                    a2[k] = __ffma2_rn(make_float2(pr[2 * k], pr[2 * k + 1]), cv2, a2[k]);
+                }
               }
             }
           }
 #pragma unroll
-          for (int gq = 0; gq < G; ++gq) pv[gq * kTile + row] = a[gq];
+          for (int gq = 0; gq < G; ++gq)
+            pv[gq * kTile + row] = (gq & 1) ? a2[gq >> 1].y : a2[gq >> 1].x;
           named_bar(2 + wg, 128);
-          if (tg == 0 && ch < r) {
-#pragma unroll
-            for (int gq = 0; gq < G; ++gq) {
-              float acc = 0.f;
-              for (int k = 0; k < TG; ++k) acc += pv[gq * kTile + k * CW + ch];
-              const int h = g * G + gq;
-              float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
-              rec[2 + ch] = acc;
+          // each (head, channel) output sums its TG partials, one output per thread
+          for (int o = row; o < vd.rank * G; o += kTile) {
+            const int gq = o / vd.rank, oc = o - gq * vd.rank;
+            const float* src = pv + gq * kTile + oc;
+            float s0 = 0.f, s1 = 0.f;
+            int k = 0;
+            for (; k + 2 <= TG; k += 2) {
+              s0 += src[k * r];
+              s1 += src[(k + 1) * r];
             }
+            if (k < TG) s0 += src[k * r];
+            const int h = g * G + gq;
+            float* rec = p.ws + (((long long)U.b * p.H + h) * p.tiles_max + U.tile) * p.rec;
+            rec[2 + oc] = s0 + s1;
           }
           if (row == 0) {
 #pragma unroll
@@ -795,7 +809,9 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
                        red[OQ * 4 + oq * 4 + 2] + red[OQ * 4 + oq * 4 + 3];
             }
           }
-          named_bar(2 + wg, 128);  // pv is reused by the next owned head
+          // pv is reused by the next owned head; after the last one, the barriers of the next
+          // chunk order these reads before the next writes
+          if (os + 1 < (HPC + 1) / 2) named_bar(2 + wg, 128);
         }
         // (8) release the value buffer
         __syncwarp();
@@ -834,7 +850,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
       }
     }
     // ---------------------------------------------------------------- dequantisers (int8/int4)
-    if (!F::kTmaA && ares) {
+    if constexpr (ares) {
       // once per tile, from the staged codes, into the resident slots
       const int tid = (warp - 12) * 32 + lane;
       const int ch = tid & 7;
@@ -995,10 +1011,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
 }
 
 // --------------------------------------------------------------------------- launchers
-template <int FMT, int HD, int G, int CG>
+template <int FMT, int HD, int G, int CG, int RES>
 static cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tmA,
                               const CUtensorMap& tmB, int grid, cudaStream_t s) {
-  auto kern = decode_split_kernel<FMT, HD, G, CG>;
+  auto kern = decode_split_kernel<FMT, HD, G, CG, RES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(p.smem_bytes));
   if (e != cudaSuccess) return e;
@@ -1025,40 +1041,45 @@ static cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tmA,
   return cudaLaunchKernelEx(&cfg, kern, p, tmA, tmB);
 }
 
-template <int FMT, int HD, int CG>
+template <int FMT, int HD, int CG, int RES>
 static cudaError_t launch_g(int G, const DecodeParams& p, const CUtensorMap& tmA,
                             const CUtensorMap& tmB, int grid, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_one<FMT, HD, 1, CG>(p, tmA, tmB, grid, s);
-    case 2: return launch_one<FMT, HD, 2, CG>(p, tmA, tmB, grid, s);
-    case 4: return launch_one<FMT, HD, 4, CG>(p, tmA, tmB, grid, s);
-    case 8: return launch_one<FMT, HD, 8, CG>(p, tmA, tmB, grid, s);
+    case 1: return launch_one<FMT, HD, 1, CG, RES>(p, tmA, tmB, grid, s);
+    case 2: return launch_one<FMT, HD, 2, CG, RES>(p, tmA, tmB, grid, s);
+    case 4: return launch_one<FMT, HD, 4, CG, RES>(p, tmA, tmB, grid, s);
+    case 8: return launch_one<FMT, HD, 8, CG, RES>(p, tmA, tmB, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int FMT, int CG>
+template <int FMT, int CG, int RES = 0>
 static cudaError_t launch_hd(int hd, int G, const DecodeParams& p, const CUtensorMap& tmA,
                              const CUtensorMap& tmB, int grid, cudaStream_t s) {
-  if (hd == 64) return launch_g<FMT, 64, CG>(G, p, tmA, tmB, grid, s);
-  if (hd == 128) return launch_g<FMT, 128, CG>(G, p, tmA, tmB, grid, s);
+  if (hd == 64) return launch_g<FMT, 64, CG, RES>(G, p, tmA, tmB, grid, s);
+  if (hd == 128) return launch_g<FMT, 128, CG, RES>(G, p, tmA, tmB, grid, s);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
                           const CUtensorMap& tmA, const CUtensorMap& tmB, int grid,
                           cudaStream_t s) {
+  const bool res = fmt == STARKV_FMT_MIXED && p.a_resident;
   if (p.cta_group == 2) {
     switch (fmt) {
       case STARKV_FMT_BF16: return launch_hd<FMT_BF16, 2>(head_dim, G, p, tmA, tmB, grid, s);
-      case STARKV_FMT_MIXED: return launch_hd<FMT_MIXED, 2>(head_dim, G, p, tmA, tmB, grid, s);
+      case STARKV_FMT_MIXED:
+        return res ? launch_hd<FMT_MIXED, 2, 1>(head_dim, G, p, tmA, tmB, grid, s)
+                   : launch_hd<FMT_MIXED, 2, 0>(head_dim, G, p, tmA, tmB, grid, s);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (fmt) {
     case STARKV_FMT_F32: return launch_hd<FMT_F32, 1>(head_dim, G, p, tmA, tmB, grid, s);
     case STARKV_FMT_BF16: return launch_hd<FMT_BF16, 1>(head_dim, G, p, tmA, tmB, grid, s);
-    case STARKV_FMT_MIXED: return launch_hd<FMT_MIXED, 1>(head_dim, G, p, tmA, tmB, grid, s);
+    case STARKV_FMT_MIXED:
+      return res ? launch_hd<FMT_MIXED, 1, 1>(head_dim, G, p, tmA, tmB, grid, s)
+                 : launch_hd<FMT_MIXED, 1, 0>(head_dim, G, p, tmA, tmB, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
