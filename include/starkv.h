@@ -130,9 +130,10 @@ typedef struct {
   int32_t n_ranges;   /* split of the KV heads of one 128-token tile into this many work
                          units; 0 = chosen from the grid size                             */
   int32_t timeout_ms; /* bound of every in-kernel wait; 0 = 4000 ms                       */
-  int32_t cta_group;  /* 0 = auto; 1 = one CTA per 128-token tile; 2 = a pair of CTAs (one
-                         cluster) per 256-token tile sharing each B_k k-block (bf16 and
-                         int8/int4 latents, 256-column chunks)                             */
+  int32_t cta_group;  /* 0 = auto (pairs for bf16 latents and for int8/int4 keys of rank
+                         <= 256, single CTAs otherwise); 1 = one CTA per 128-token tile;
+                         2 = a pair of CTAs (one cluster) per 256-token tile sharing each
+                         B_k k-block (bf16 and int8/int4 latents, 256-column chunks)       */
 } starkv_decode_opts;
 
 /* Fill ``out`` from ``cfg``: per-latent mixed split, block offsets, page size.

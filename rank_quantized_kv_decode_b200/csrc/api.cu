@@ -489,7 +489,11 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   const bool pair_ok = fmt != STARKV_FMT_F32 && p.NC == 256 && info.sms >= 2;
   if (want_cg == 2 && !pair_ok)
     return fail(STARKV_ERR_UNSUPPORTED, "CTA pairs need bf16 or int8/int4 latents and 256-column chunks");
-  p.cta_group = (want_cg == 1 || !pair_ok) ? 1 : 2;
+  // the streamed int8/int4 operand (key rank > 256, dequantised per ring stage) ran slower on
+  // pairs than on single CTAs (10.1 vs 12.0 ms at batch 16, context 16384, rank 1024): the
+  // default keeps single-CTA tiles there
+  const bool pair_default = pair_ok && !(fmt == STARKV_FMT_MIXED && p.kb_count > 4);
+  p.cta_group = want_cg == 2 ? 2 : (want_cg == 1 ? 1 : (pair_default ? 2 : 1));
   const int CG = p.cta_group;
   int grid_cap = info.sms;
   if (opts && opts->max_ctas > 0 && opts->max_ctas < grid_cap) grid_cap = opts->max_ctas;
@@ -534,12 +538,26 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   }
   for (int g = 0; g < c.n_kv_heads; ++g) p.vh[g] = lat_desc(lay->seg[1 + g]);
 
-  // int8/int4 keys of rank <= 256 keep the dequantised tile resident for all its chunks
-  const bool ares = fmt == STARKV_FMT_MIXED && p.kb_count <= 4;
-  p.a_resident = ares ? 1 : 0;
+  // int8/int4 keys: of rank <= 256, the dequantised tile stays resident for all its chunks
+  // (mode 1, codes double-buffered); above that, the tile's codes are staged in shared memory
+  // once and the operand is streamed through the ring (mode 2, one code buffer) when they
+  // fit, else the dequantisers read the codes from global memory (mode 0)
+  int modes[2] = {0, 0};
+  int n_modes = 1;
+  if (fmt == STARKV_FMT_MIXED) {
+    if (p.kb_count <= 4) {
+      modes[0] = 1;
+    } else {
+      modes[0] = 2;
+      modes[1] = 0;
+      n_modes = 2;
+    }
+  }
+  int key_region = 0;
   {
     const starkv_segment& k = lay->seg[0];
-    p.key_region = ares ? static_cast<int>(k.off_sc + int64_t(kPage) * 2 * (k.g8 + k.g4) - k.off_i8) : 0;
+    if (fmt == STARKV_FMT_MIXED)
+      key_region = static_cast<int>(k.off_sc + int64_t(kPage) * 2 * (k.g8 + k.g4) - k.off_i8);
   }
   // shared-memory plan: ring stages of (A k-block, B k-block), value buffers, small arrays
   p.vslot = (vmax + 127) / 128 * 128;
@@ -547,7 +565,11 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   const size_t limit = std::min<size_t>(decode_smem_limit(), info.smem_optin);
   bool planned = false;
   const int plans[][2] = {{6, 2}, {6, 1}, {5, 2}, {5, 1}, {4, 2}, {4, 1}, {3, 2}, {3, 1}, {2, 1}};
+  for (int mi = 0; mi < n_modes && !planned; ++mi)
   for (const auto& pl : plans) {
+    const int mode = modes[mi];
+    const bool ares = mode == 1;
+    const int ncb = mode == 1 ? 2 : (mode == 2 ? 1 : 0);  // code buffers
     size_t off = 0;
     const int S = pl[0], NVB = pl[1];
     const size_t split = fmt == STARKV_FMT_F32 ? 2 : 1;  // hi/lo copies for 3xTF32
@@ -555,7 +577,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     const size_t off_b = off;
     off += S * split * bstage;
     const size_t off_codes = off;
-    off += ares ? 2 * 2 * static_cast<size_t>(p.key_region) : 0;
+    off += static_cast<size_t>(ncb) * 2 * static_cast<size_t>(key_region);
     const size_t off_v = off;
     off += static_cast<size_t>(NVB) * 2 * p.vslot;
     const size_t QPC = static_cast<size_t>(256 / d) * p.G;  // query heads of a full chunk
@@ -579,6 +601,8 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     // (each CTA allocates all 512 TMEM columns)
     const size_t total = std::max<size_t>(off + 1024, 120 * 1024);
     if (total <= limit) {
+      p.a_resident = mode;
+      p.key_region = mode ? key_region : 0;
       p.stages = S;
       p.nvb = NVB;
       p.off_b = static_cast<uint32_t>(off_b);

@@ -137,7 +137,9 @@ __device__ __forceinline__ float vchan_load(const uint8_t* slot, const VChan& v,
     const unsigned b = slot[v.off + row * v.stride];
     const int q = static_cast<int>(b << v.lsh) >> v.rsh;
     const float s = __half2float(*reinterpret_cast<const __half*>(slot + v.soff + row * v.sstride));
-    return s * static_cast<float>(q);
+    // q as a float without the conversion unit: 1.5 * 2^23 + q has an ulp of 1, so its bits
+    // are those of 1.5 * 2^23 plus q, and one subtraction leaves q exactly
+    return s * (__int_as_float(0x4B400000 + q) - 12582912.0f);
   }
 }
 
@@ -182,52 +184,104 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) {
+  __half2 h;
+  memcpy(&h, &u, 4);
+  return h;
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+  uint32_t u;
+  memcpy(&u, &h, 4);
+  return u;
+}
 
 // Channels [k0, k0+8) of token row ``prow`` of a page whose key blocks are at ``base`` + the
 // offsets of ``kd`` (the page itself in global memory, or a copy of its key region in shared
-// memory with the offsets rebased).
+// memory with the offsets rebased), one channel at a time: the ragged edges of the int8 and
+// int4 parts.
 __device__ __forceinline__ uint4 dequant8_at(const uint8_t* base, const LatDesc& kd, int prow, int k0) {
-  uint4 z = make_uint4(0, 0, 0, 0);
-  if (k0 >= kd.rank) return z;
   float v[8];
-  if (k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(base + kd.off0 + prow * kd.n8 + k0);
-    const float s = __half2float(reinterpret_cast<const __half*>(base + kd.off2)[prow * kd.ng + (k0 >> 5)]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[e] = s * static_cast<float>(static_cast<int8_t>((raw.x >> (8 * e)) & 0xFF));
-      v[4 + e] = s * static_cast<float>(static_cast<int8_t>((raw.y >> (8 * e)) & 0xFF));
-    }
-  } else if (k0 >= kd.n8 && ((k0 - kd.n8) & 7) == 0 && k0 + 8 <= kd.rank && (kd.nb4 & 3) == 0) {
-    const int j0 = k0 - kd.n8;
-    const uint32_t raw = *reinterpret_cast<const uint32_t*>(base + kd.off1 + prow * kd.nb4 + (j0 >> 1));
-    const float s =
-        __half2float(reinterpret_cast<const __half*>(base + kd.off2)[prow * kd.ng + kd.g8 + (j0 >> 5)]);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int nib = (raw >> (4 * e)) & 15;
-      v[e] = s * static_cast<float>((nib ^ 8) - 8);
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int k = k0 + e;
-      v[e] = k < kd.rank ? key_code_value(base, kd, prow, k) : 0.f;
-    }
+  for (int e = 0; e < 8; ++e) {
+    const int k = k0 + e;
+    v[e] = k < kd.rank ? key_code_value(base, kd, prow, k) : 0.f;
   }
-  z.x = pack_h2(v[0], v[1]);
-  z.y = pack_h2(v[2], v[3]);
-  z.z = pack_h2(v[4], v[5]);
-  z.w = pack_h2(v[6], v[7]);
-  return z;
+  return make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]),
+                    pack_h2(v[6], v[7]));
 }
 
-// Row r of the tile's operand, read from the pages in global memory.
-__device__ __forceinline__ uint4 dequant8(const DecodeParams& p, const Unit& U, int r, int k0) {
-  const int pp = r >> 6, prow = r & 63;
-  const int pg = U.page(pp);
-  if (pg < 0 || r >= U.nvalid) return make_uint4(0, 0, 0, 0);
-  return dequant8_at(p.cache + (long long)pg * p.page_bytes, p.key, prow, k0);
+// Channels [k0, k0+8) of the 8 tile rows r = row0 + 16 it (it < 8), as fp16 into the
+// 128-byte-swizzled operand stage ``dst``.  ``key_base(r)`` gives the key blocks of row r's
+// page (or nullptr for a row past the sequence or on a missing page, stored as zeros).  All
+// code loads are issued before the first store: the stores go to shared memory too, so the
+// compiler could not move a later row's load above an earlier row's store.
+template <class BaseFn>
+__device__ __forceinline__ void dequant_rows8(uint8_t* dst, const LatDesc& kd, int k0, int ch,
+                                              int row0, BaseFn key_base) {
+  const bool i8 = k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0;
+  const bool i4 = !i8 && k0 >= kd.n8 && ((k0 - kd.n8) & 7) == 0 && k0 + 8 <= kd.rank &&
+                  (kd.nb4 & 3) == 0;
+  if (i8 || i4) {
+    const int j0 = k0 - kd.n8;
+    const int coff = i8 ? kd.off0 + k0 : kd.off1 + (j0 >> 1);
+    const int cpitch = i8 ? kd.n8 : kd.nb4;
+    const int soff = kd.off2 + 2 * (i8 ? (k0 >> 5) : kd.g8 + (j0 >> 5));
+    uint32_t cx[8], cy[8];
+    unsigned short sb[8];
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int r = row0 + 16 * it;
+      const uint8_t* b = key_base(r);
+      cx[it] = 0u;
+      cy[it] = 0u;
+      sb[it] = 0;
+      if (b) {
+        const int prow = r & 63;
+        if (i8) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(b + coff + prow * cpitch);
+          cx[it] = raw.x;
+          cy[it] = raw.y;
+        } else {
+          cx[it] = *reinterpret_cast<const uint32_t*>(b + coff + prow * cpitch);
+        }
+        sb[it] = *reinterpret_cast<const unsigned short*>(b + soff + prow * 2 * kd.ng);
+      }
+    }
+    // In fp16 pairs: a code c becomes the fp16 value 1024 + (c + bias) by placing c + bias in
+    // the mantissa under the exponent bits 0x64 (bias 128 for int8, 8 for int4), one
+    // subtraction recovers c exactly, and one multiplication by the fp16 scale rounds s*c once
+    // -- the value of rounding the exact fp32 product s*c to fp16.
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const __half2 s2 = __half2half2(__ushort_as_half(sb[it]));
+      uint4 z;
+      if (i8) {
+        const uint32_t bx = cx[it] ^ 0x80808080u, by = cy[it] ^ 0x80808080u;
+        const __half2 off = __half2half2(__ushort_as_half(0x6480));  // 1152
+        z.x = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(bx, 0x64646464u, 0x4140)), off), s2));
+        z.y = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(bx, 0x64646464u, 0x4342)), off), s2));
+        z.z = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(by, 0x64646464u, 0x4140)), off), s2));
+        z.w = h2_bits(__hmul2(__hsub2(bits_h2(__byte_perm(by, 0x64646464u, 0x4342)), off), s2));
+      } else {
+        const uint32_t raw = cx[it], hi = raw >> 4;
+        const __half2 off = __half2half2(__ushort_as_half(0x6408));  // 1032
+        z.x = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0400) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+        z.y = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0501) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+        z.z = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0602) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+        z.w = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0703) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+      }
+      *reinterpret_cast<uint4*>(dst + sw128_offset(row0 + 16 * it, ch)) = z;
+    }
+  } else {
+    // ragged edges of the int8 / int4 parts
+#pragma unroll 2
+    for (int it = 0; it < 8; ++it) {
+      const int r = row0 + 16 * it;
+      const uint8_t* b = key_base(r);
+      const uint4 z = b ? dequant8_at(b, kd, r & 63, k0) : make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch)) = z;
+    }
+  }
 }
 
 template <int FMT>
@@ -278,8 +332,13 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   // resident operand (int8/int4 keys of rank <= 256): dequantised once per tile into kb_count
   // slots, each used by every chunk of the unit; the tile's codes are staged by bulk copy
   const int B_AF = B_TD + 1, B_AE = B_AF + 4, B_CF = B_AE + 4, B_CE = B_CF + 2;
-  constexpr bool ares = RES != 0;  // resident operand (int8/int4 keys of rank <= 256)
-  uint8_t* sCodes = smem + p.off_codes;  // [2 buffers][2 pages][key_region]
+  // int8/int4 keys: RES 1 = operand dequantised once per tile and kept resident (rank <= 256);
+  // RES 2 = the tile's codes staged in shared memory, operand streamed per ring stage; RES 0 =
+  // operand streamed from the codes in global memory
+  constexpr bool ares = RES == 1;
+  constexpr bool staged = RES != 0;
+  constexpr int NCB = RES == 1 ? 2 : 1;  // code buffers
+  uint8_t* sCodes = smem + p.off_codes;  // [NCB buffers][2 pages][key_region]
   // misc: [0] TMEM base, [1] abort flag, [2..3] per-warpgroup stop snapshots
   uint32_t* misc = reinterpret_cast<uint32_t*>(bars + B_CE + 2);
   auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -489,7 +548,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
     }
   } else if (warp == 3) {
     // ---------------------------------------------------------------- key-code stager
-    if (ares && lane == 0) {
+    if (staged && lane == 0) {
       const uint32_t kreg = static_cast<uint32_t>(p.key_region);
       int cb = 0;
       uint32_t cph = 0, issued = 0, last_phase = 0;
@@ -507,7 +566,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         }
         issued |= 1u << cb;
         last_phase = (last_phase & ~(1u << cb)) | (cph << cb);
-        if (++cb == 2) { cb = 0; cph ^= 1u; }
+        if (++cb == NCB) { cb = 0; cph ^= 1u; }
       }
       for (int k = 0; k < 2; ++k)
         if (issued & (1u << k)) wait_drain(bar(B_CF + k), (last_phase >> k) & 1u, p.timeout_ns);
@@ -871,15 +930,10 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             ok = false;
             break;
           }
-          uint8_t* dst = sA + kb * kAStage;
-#pragma unroll 2
-          for (int it = 0; it < 8; ++it) {
-            const int r = it * 16 + (tid >> 3);
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (r < U.nvalid && U.page(r >> 6) >= 0)
-              v = dequant8_at(sCodes + (cb * 2 + (r >> 6)) * kreg, kd, r & 63, kb * 64 + ch * 8);
-            *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch)) = v;
-          }
+          const uint8_t* codes = sCodes + cb * 2 * kreg;
+          dequant_rows8(sA + kb * kAStage, kd, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) {
+            return (r < U.nvalid && U.page(r >> 6) >= 0) ? codes + (r >> 6) * kreg : nullptr;
+          });
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -895,13 +949,24 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
         if (++cb == 2) { cb = 0; cph ^= 1u; }
       }
     } else if constexpr (!F::kTmaA) {
+      // streamed operand, one ring stage per (chunk, k-block): from the tile's codes staged in
+      // shared memory (RES 2) or from the pages in global memory (RES 0)
       const int tid = (warp - 12) * 32 + lane;
+      const int ch = tid & 7;
+      LatDesc kd = p.key;  // offsets rebased onto the staged key region
+      kd.off1 -= kd.off0;
+      kd.off2 -= kd.off0;
+      kd.off0 = 0;
+      const int kreg = p.key_region;
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t phase = 0, cph = 0;
       bool ok = true;
       for (int u = unit0; ok && u < p.total_units; u += unit_step) {
         Unit U;
         if (!get_unit<CG>(p, u, U, false, crank)) continue;
+        if constexpr (staged) {
+          if (!__all_sync(0xffffffffu, wait_bounded(bar(B_CF), cph, wc))) break;
+        }
         for (int c = U.c0; ok && c < U.c1; ++c) {
           for (int kb = 0; kb < p.kb_count; ++kb) {
             // warp-uniform decision (the __syncwarp below needs every lane)
@@ -910,12 +975,15 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
               break;
             }
             uint8_t* dst = sA + stage * kAStage;
-            const int ch = tid & 7;
-#pragma unroll 2
-            for (int it = 0; it < 8; ++it) {
-              const int r = it * 16 + (tid >> 3);
-              const uint4 v = dequant8(p, U, r, kb * 64 + ch * 8);
-              *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch)) = v;
+            if constexpr (staged) {
+              dequant_rows8(dst, kd, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) {
+                return (r < U.nvalid && U.page(r >> 6) >= 0) ? sCodes + (r >> 6) * kreg : nullptr;
+              });
+            } else {
+              dequant_rows8(dst, p.key, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) -> const uint8_t* {
+                const int pg = U.page(r >> 6);
+                return (r < U.nvalid && pg >= 0) ? p.cache + (long long)pg * p.page_bytes : nullptr;
+              });
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -927,6 +995,12 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             }
             if (++stage == S) { stage = 0; phase ^= 1u; }
           }
+        }
+        if constexpr (staged) {
+          // the staged codes may be overwritten once every chunk of the unit has used them
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_CE));
+          cph ^= 1u;
         }
       }
     }
@@ -1064,13 +1138,14 @@ static cudaError_t launch_hd(int hd, int G, const DecodeParams& p, const CUtenso
 cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
                           const CUtensorMap& tmA, const CUtensorMap& tmB, int grid,
                           cudaStream_t s) {
-  const bool res = fmt == STARKV_FMT_MIXED && p.a_resident;
+  const int res = fmt == STARKV_FMT_MIXED ? p.a_resident : 0;
   if (p.cta_group == 2) {
     switch (fmt) {
       case STARKV_FMT_BF16: return launch_hd<FMT_BF16, 2>(head_dim, G, p, tmA, tmB, grid, s);
       case STARKV_FMT_MIXED:
-        return res ? launch_hd<FMT_MIXED, 2, 1>(head_dim, G, p, tmA, tmB, grid, s)
-                   : launch_hd<FMT_MIXED, 2, 0>(head_dim, G, p, tmA, tmB, grid, s);
+        return res == 1   ? launch_hd<FMT_MIXED, 2, 1>(head_dim, G, p, tmA, tmB, grid, s)
+               : res == 2 ? launch_hd<FMT_MIXED, 2, 2>(head_dim, G, p, tmA, tmB, grid, s)
+                          : launch_hd<FMT_MIXED, 2, 0>(head_dim, G, p, tmA, tmB, grid, s);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -1078,8 +1153,9 @@ cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
     case STARKV_FMT_F32: return launch_hd<FMT_F32, 1>(head_dim, G, p, tmA, tmB, grid, s);
     case STARKV_FMT_BF16: return launch_hd<FMT_BF16, 1>(head_dim, G, p, tmA, tmB, grid, s);
     case STARKV_FMT_MIXED:
-      return res ? launch_hd<FMT_MIXED, 1, 1>(head_dim, G, p, tmA, tmB, grid, s)
-                 : launch_hd<FMT_MIXED, 1, 0>(head_dim, G, p, tmA, tmB, grid, s);
+      return res == 1   ? launch_hd<FMT_MIXED, 1, 1>(head_dim, G, p, tmA, tmB, grid, s)
+             : res == 2 ? launch_hd<FMT_MIXED, 1, 2>(head_dim, G, p, tmA, tmB, grid, s)
+                        : launch_hd<FMT_MIXED, 1, 0>(head_dim, G, p, tmA, tmB, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -62,7 +62,7 @@ struct DecodeParams {
   int H, Hkv, G, d, rk, key_rank_cols;
   int NC, n_chunks, n_ranges, cpr, kb_count, total_units;
   int cta_group;  // 1: one CTA per 128-token tile; 2: a CTA pair per 256-token tile
-  int a_resident;  // int8/int4 keys: operand dequantised once per tile (kb_count <= 4)
+  int a_resident;  // int8/int4 keys: 1 = operand resident per tile, 2 = codes staged per tile, 0 = neither
   int key_region;  // bytes of the key blocks of one page (int8 | int4 | scales)
   uint32_t idesc;
   float qscale;  // log2(e) / sqrt(d)

@@ -121,3 +121,19 @@ def test_bad_block_table_entry_is_flagged():
     finally:
         wl.block_table.copy_(saved)
         wl.lc.status.zero_()
+
+
+def test_key_codes_too_large_to_stage_read_from_global_memory():
+    """int8/int4 keys of rank 2048: a 128-token tile's codes (2 x 90 KB) do not fit in shared
+    memory next to the ring, so the dequantisers read them from the pages in global memory;
+    ranks up to ~1024 stage them (the other cases of this file)."""
+    from oracle.workloads import Ref
+    from rank_quantized_kv_decode_b200 import synth
+
+    ov = dict(key_rank=2048, batch=1, context=200)
+    wl = W.build(3, seq_lens=[200], **ov)
+    W.decode(wl)
+    torch.cuda.synchronize()
+    assert wl.lc.status.item() == 0
+    ref = Ref(synth.workload(3, **ov), False)
+    tolerance_check(wl.out[0].cpu().numpy(), ref.expected(0, 200))
