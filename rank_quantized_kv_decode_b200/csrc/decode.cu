@@ -211,12 +211,15 @@ __device__ __forceinline__ uint4 dequant8_at(const uint8_t* base, const LatDesc&
 }
 
 // Channels [k0, k0+8) of the 8 tile rows r = row0 + 16 it (it < 8), as fp16 into the
-// 128-byte-swizzled operand stage ``dst``.  ``key_base(r)`` gives the key blocks of row r's
-// page (or nullptr for a row past the sequence or on a missing page, stored as zeros).  All
-// code loads are issued before the first store: the stores go to shared memory too, so the
-// compiler could not move a later row's load above an earlier row's store.
-template <class BaseFn>
-__device__ __forceinline__ void dequant_rows8(uint8_t* dst, const LatDesc& kd, int k0, int ch,
+// 128-byte-swizzled operand stage at shared address ``dst``.  ``key_base(r)`` gives the key
+// blocks of row r's page: a 32-bit shared address (``kNoRow`` for a row past the sequence or
+// on a missing page) when SMEM, else a global pointer (nullptr for such a row); those rows are
+// stored as zeros.  All code loads are issued before the first store: the stores go to shared
+// memory, so the compiler could not move a later row's load above an earlier row's store.
+constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+
+template <bool SMEM, class BaseFn>
+__device__ __forceinline__ void dequant_rows8(uint32_t dst, const LatDesc& kd, int k0, int ch,
                                               int row0, BaseFn key_base) {
   const bool i8 = k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0;
   const bool i4 = !i8 && k0 >= kd.n8 && ((k0 - kd.n8) & 7) == 0 && k0 + 8 <= kd.rank &&
@@ -231,20 +234,34 @@ __device__ __forceinline__ void dequant_rows8(uint8_t* dst, const LatDesc& kd, i
 #pragma unroll
     for (int it = 0; it < 8; ++it) {
       const int r = row0 + 16 * it;
-      const uint8_t* b = key_base(r);
+      const int prow = r & 63;
+      const auto b = key_base(r);
       cx[it] = 0u;
       cy[it] = 0u;
       sb[it] = 0;
-      if (b) {
-        const int prow = r & 63;
-        if (i8) {
-          const uint2 raw = *reinterpret_cast<const uint2*>(b + coff + prow * cpitch);
-          cx[it] = raw.x;
-          cy[it] = raw.y;
-        } else {
-          cx[it] = *reinterpret_cast<const uint32_t*>(b + coff + prow * cpitch);
+      if constexpr (SMEM) {
+        if (b != kNoRow) {
+          const uint32_t a = b + coff + prow * cpitch;
+          if (i8) {
+            const uint2 raw = ld_shared_v2(a);
+            cx[it] = raw.x;
+            cy[it] = raw.y;
+          } else {
+            cx[it] = ld_shared_u32(a);
+          }
+          sb[it] = ld_shared_u16(b + soff + prow * 2 * kd.ng);
         }
-        sb[it] = *reinterpret_cast<const unsigned short*>(b + soff + prow * 2 * kd.ng);
+      } else {
+        if (b) {
+          if (i8) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(b + coff + prow * cpitch);
+            cx[it] = raw.x;
+            cy[it] = raw.y;
+          } else {
+            cx[it] = *reinterpret_cast<const uint32_t*>(b + coff + prow * cpitch);
+          }
+          sb[it] = *reinterpret_cast<const unsigned short*>(b + soff + prow * 2 * kd.ng);
+        }
       }
     }
     // In fp16 pairs: a code c becomes the fp16 value 1024 + (c + bias) by placing c + bias in
@@ -270,16 +287,21 @@ __device__ __forceinline__ void dequant_rows8(uint8_t* dst, const LatDesc& kd, i
         z.z = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0602) & 0x000F000Fu) ^ 0x64086408u), off), s2));
         z.w = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0703) & 0x000F000Fu) ^ 0x64086408u), off), s2));
       }
-      *reinterpret_cast<uint4*>(dst + sw128_offset(row0 + 16 * it, ch)) = z;
+      st_shared_v4(dst + sw128_offset(row0 + 16 * it, ch), z);
     }
   } else {
-    // ragged edges of the int8 / int4 parts
+    // ragged edges of the int8 / int4 parts, one channel at a time (generic accesses)
 #pragma unroll 2
     for (int it = 0; it < 8; ++it) {
       const int r = row0 + 16 * it;
-      const uint8_t* b = key_base(r);
-      const uint4 z = b ? dequant8_at(b, kd, r & 63, k0) : make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(dst + sw128_offset(r, ch)) = z;
+      const auto b = key_base(r);
+      uint4 z = make_uint4(0, 0, 0, 0);
+      if constexpr (SMEM) {
+        if (b != kNoRow) z = dequant8_at(smem_generic(b), kd, r & 63, k0);
+      } else {
+        if (b) z = dequant8_at(b, kd, r & 63, k0);
+      }
+      st_shared_v4(dst + sw128_offset(r, ch), z);
     }
   }
 }
@@ -930,10 +952,13 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             ok = false;
             break;
           }
-          const uint8_t* codes = sCodes + cb * 2 * kreg;
-          dequant_rows8(sA + kb * kAStage, kd, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) {
-            return (r < U.nvalid && U.page(r >> 6) >= 0) ? codes + (r >> 6) * kreg : nullptr;
-          });
+          const uint32_t codes = smem_u32(sCodes) + static_cast<uint32_t>(cb * 2 * kreg);
+          dequant_rows8<true>(smem_u32(sA + kb * kAStage), kd, kb * 64 + ch * 8, ch, tid >> 3,
+                              [&](int r) -> uint32_t {
+                                return (r < U.nvalid && U.page(r >> 6) >= 0)
+                                           ? codes + static_cast<uint32_t>((r >> 6) * kreg)
+                                           : kNoRow;
+                              });
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -974,13 +999,16 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
               ok = false;
               break;
             }
-            uint8_t* dst = sA + stage * kAStage;
+            const uint32_t dst = smem_u32(sA + stage * kAStage);
             if constexpr (staged) {
-              dequant_rows8(dst, kd, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) {
-                return (r < U.nvalid && U.page(r >> 6) >= 0) ? sCodes + (r >> 6) * kreg : nullptr;
+              const uint32_t codes = smem_u32(sCodes);
+              dequant_rows8<true>(dst, kd, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) -> uint32_t {
+                return (r < U.nvalid && U.page(r >> 6) >= 0)
+                           ? codes + static_cast<uint32_t>((r >> 6) * kreg)
+                           : kNoRow;
               });
             } else {
-              dequant_rows8(dst, p.key, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) -> const uint8_t* {
+              dequant_rows8<false>(dst, p.key, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) -> const uint8_t* {
                 const int pg = U.page(r >> 6);
                 return (r < U.nvalid && pg >= 0) ? p.cache + (long long)pg * p.page_bytes : nullptr;
               });
