@@ -211,8 +211,8 @@ __device__ __forceinline__ uint4 dequant8_at(const uint8_t* base, const LatDesc&
 }
 
 // Channels [k0, k0+8) of the 8 tile rows r = row0 + 16 it (it < 8), as fp16 into the
-// 128-byte-swizzled operand stage at shared address ``dst``.  ``key_base(r)`` gives the key
-// blocks of row r's page: a 32-bit shared address (``kNoRow`` for a row past the sequence or
+// 128-byte-swizzled operand stage at shared address ``dst`` (row0 < 16, so rows it < 4 lie on
+// the tile's first page).  ``key_base(it, r)`` gives the key blocks of row r's page: a 32-bit shared address (``kNoRow`` for a row past the sequence or
 // on a missing page) when SMEM, else a global pointer (nullptr for such a row); those rows are
 // stored as zeros.  All code loads are issued before the first store: the stores go to shared
 // memory, so the compiler could not move a later row's load above an earlier row's store.
@@ -235,7 +235,7 @@ __device__ __forceinline__ void dequant_rows8(uint32_t dst, const LatDesc& kd, i
     for (int it = 0; it < 8; ++it) {
       const int r = row0 + 16 * it;
       const int prow = r & 63;
-      const auto b = key_base(r);
+      const auto b = key_base(it, r);
       cx[it] = 0u;
       cy[it] = 0u;
       sb[it] = 0;
@@ -294,7 +294,7 @@ __device__ __forceinline__ void dequant_rows8(uint32_t dst, const LatDesc& kd, i
 #pragma unroll 2
     for (int it = 0; it < 8; ++it) {
       const int r = row0 + 16 * it;
-      const auto b = key_base(r);
+      const auto b = key_base(it, r);
       uint4 z = make_uint4(0, 0, 0, 0);
       if constexpr (SMEM) {
         if (b != kNoRow) z = dequant8_at(smem_generic(b), kd, r & 63, k0);
@@ -953,11 +953,11 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             break;
           }
           const uint32_t codes = smem_u32(sCodes) + static_cast<uint32_t>(cb * 2 * kreg);
+          const uint32_t pb0 = U.page0 >= 0 ? codes : kNoRow;
+          const uint32_t pb1 = U.page1 >= 0 ? codes + static_cast<uint32_t>(kreg) : kNoRow;
           dequant_rows8<true>(smem_u32(sA + kb * kAStage), kd, kb * 64 + ch * 8, ch, tid >> 3,
-                              [&](int r) -> uint32_t {
-                                return (r < U.nvalid && U.page(r >> 6) >= 0)
-                                           ? codes + static_cast<uint32_t>((r >> 6) * kreg)
-                                           : kNoRow;
+                              [&](int it, int r) -> uint32_t {
+                                return r < U.nvalid ? (it < 4 ? pb0 : pb1) : kNoRow;
                               });
           fence_proxy_async_smem();
           __syncwarp();
@@ -1002,16 +1002,19 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
             const uint32_t dst = smem_u32(sA + stage * kAStage);
             if constexpr (staged) {
               const uint32_t codes = smem_u32(sCodes);
-              dequant_rows8<true>(dst, kd, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) -> uint32_t {
-                return (r < U.nvalid && U.page(r >> 6) >= 0)
-                           ? codes + static_cast<uint32_t>((r >> 6) * kreg)
-                           : kNoRow;
-              });
+              const uint32_t pb0 = U.page0 >= 0 ? codes : kNoRow;
+              const uint32_t pb1 = U.page1 >= 0 ? codes + static_cast<uint32_t>(kreg) : kNoRow;
+              dequant_rows8<true>(dst, kd, kb * 64 + ch * 8, ch, tid >> 3,
+                                  [&](int it, int r) -> uint32_t {
+                                    return r < U.nvalid ? (it < 4 ? pb0 : pb1) : kNoRow;
+                                  });
             } else {
-              dequant_rows8<false>(dst, p.key, kb * 64 + ch * 8, ch, tid >> 3, [&](int r) -> const uint8_t* {
-                const int pg = U.page(r >> 6);
-                return (r < U.nvalid && pg >= 0) ? p.cache + (long long)pg * p.page_bytes : nullptr;
-              });
+              const uint8_t* gb0 = U.page0 >= 0 ? p.cache + (long long)U.page0 * p.page_bytes : nullptr;
+              const uint8_t* gb1 = U.page1 >= 0 ? p.cache + (long long)U.page1 * p.page_bytes : nullptr;
+              dequant_rows8<false>(dst, p.key, kb * 64 + ch * 8, ch, tid >> 3,
+                                   [&](int it, int r) -> const uint8_t* {
+                                     return r < U.nvalid ? (it < 4 ? gb0 : gb1) : nullptr;
+                                   });
             }
             fence_proxy_async_smem();
             __syncwarp();
