@@ -1084,19 +1084,34 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   if (lane == 0) s_m[warp] = m;
   __syncthreads();
   const float M = fmaxf(fmaxf(s_m[0], s_m[1]), fmaxf(s_m[2], s_m[3]));
-  // each warp takes every 4th tile; lanes cover the latent channels
+  // each warp takes every 4th tile, eight tiles per batch with all their loads issued first;
+  // lanes cover the latent channels
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float lsum = 0.f;
-  for (int t = warp; t < T; t += 4) {
-    const float* rc = recs + (long long)t * p.rec;
-    const float lt = rc[1];
-    if (!(lt > 0.f)) continue;
-    const float w = exp2f(rc[0] - M);
-    lsum += lt * w;
+  for (int tb = warp; tb < T; tb += 32) {
+    float mm[8], ll[8], vv[8][4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int i = lane + 32 * k;
-      if (i < r) acc[k] = fmaf(rc[2 + i], w, acc[k]);
+    for (int jj = 0; jj < 8; ++jj) {
+      const int t = tb + 4 * jj;
+      const bool ok = t < T;
+      const float* rc = recs + (long long)(ok ? t : tb) * p.rec;
+      mm[jj] = ok ? rc[0] : 0.f;
+      ll[jj] = ok ? rc[1] : 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = lane + 32 * k;
+        vv[jj][k] = (ok && i < r) ? rc[2 + i] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      // a tile without weight (none, or a garbage record) contributes nothing
+      const float w = ll[jj] > 0.f ? exp2f(mm[jj] - M) : 0.f;
+      if (w > 0.f) {
+        lsum += ll[jj] * w;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = fmaf(vv[jj][k], w, acc[k]);
+      }
     }
   }
 #pragma unroll
@@ -1105,13 +1120,23 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   __syncthreads();
   const float l = s_acc[0][128] + s_acc[1][128] + s_acc[2][128] + s_acc[3][128];
   const float inv = l > 0.f ? 1.f / l : 0.f;
-  if (tid < r) s_a[tid] = (s_acc[0][tid] + s_acc[1][tid] + s_acc[2][tid] + s_acc[3][tid]) * inv;
+  s_a[tid] = tid < r ? (s_acc[0][tid] + s_acc[1][tid] + s_acc[2][tid] + s_acc[3][tid]) * inv : 0.f;
   __syncthreads();
+  // o_c = sum_i a_i B_v[i][c], 32 rows of B_v in flight at a time (a_i = 0 for i >= r)
   const float* Bv = p.Bv + (long long)(vd.col - p.key_rank_cols) * p.d;
   for (int c = tid; c < p.d; c += 128) {
-    float o = 0.f;
-    for (int i = 0; i < r; ++i) o = fmaf(s_a[i], Bv[(long long)i * p.d + c], o);
-    outp[c] = o;
+    float o0 = 0.f, o1 = 0.f;
+    for (int i0 = 0; i0 < r; i0 += 32) {
+      float bv[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) bv[k] = i0 + k < r ? __ldg(Bv + (long long)(i0 + k) * p.d + c) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; k += 2) {
+        o0 = fmaf(s_a[i0 + k], bv[k], o0);
+        o1 = fmaf(s_a[i0 + k + 1], bv[k + 1], o1);
+      }
+    }
+    outp[c] = o0 + o1;
   }
 }
 

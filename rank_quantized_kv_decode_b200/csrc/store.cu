@@ -53,20 +53,18 @@ __device__ __forceinline__ TokenSlot locate(const StoreParams& p, int n, int li,
   return t;
 }
 
-// Sum of the split-K partials of one value, in split order (deterministic).  The loads are
-// issued before the adds so they are in flight together.
+// Sum of the split-K partials of one value, in split order (deterministic).  Up to 16 loads
+// are issued before the first add, so a decode step's partials arrive in one round trip.
 __device__ __forceinline__ float split_sum(const float* src, long long stride, int nsplit) {
-  float v = src[0];
-  int s = 1;
-  for (; s + 4 <= nsplit; s += 4) {
-    const float a = src[s * stride], b = src[(s + 1) * stride];
-    const float c = src[(s + 2) * stride], d = src[(s + 3) * stride];
-    v += a;
-    v += b;
-    v += c;
-    v += d;
+  float v = 0.f;
+  for (int s0 = 0; s0 < nsplit; s0 += 16) {
+    float t[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) t[k] = s0 + k < nsplit ? __ldcg(src + (s0 + k) * stride) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (s0 + k < nsplit) v = (s0 + k == 0) ? t[k] : v + t[k];
   }
-  for (; s < nsplit; ++s) v += src[s * stride];
   return v;
 }
 
@@ -82,16 +80,22 @@ __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ Stor
   while (p.chunk_start[li + 1] <= ck) ++li;
   const int cl = ck - p.chunk_start[li];  // chunk within the latent
   const LatDesc& d = p.lat[li];
-  const TokenSlot ts = locate(p, n, (li == 0 && cl == 0) ? 0 : 1, lane);
   const float* src = p.src + (long long)n * p.proj_cols + d.col;
   float* lout = p.latents_out ? p.latents_out + (long long)n * p.proj_cols + d.col : nullptr;
+  // this lane's channel of the chunk; the partial sums are loaded before the page lookup so
+  // that both round trips overlap
+  const bool plain = p.fmt == STARKV_FMT_F32 || p.fmt == STARKV_FMT_BF16;
+  const bool is8 = !plain && cl < d.g8;
+  const int n4 = d.rank - d.n8;
+  const int j = (plain || is8) ? 0 : (cl - d.g8) * 32 + lane;  // int4 channel index
+  const int i = (plain || is8) ? cl * 32 + lane : d.n8 + j;    // channel in the latent
+  const bool in = plain ? i < d.rank : (is8 ? i < d.n8 : j < n4);
+  const float c = in ? split_sum(src + i, p.split_stride, p.nsplit) : 0.f;
+  if (lout && in) lout[i] = c;
+  const TokenSlot ts = locate(p, n, (li == 0 && cl == 0) ? 0 : 1, lane);
 
-  if (p.fmt == STARKV_FMT_F32 || p.fmt == STARKV_FMT_BF16) {
-    const int i = cl * 32 + lane;
-    if (i >= d.rank) return;
-    const float c = split_sum(src + i, p.split_stride, p.nsplit);
-    if (lout) lout[i] = c;
-    if (!ts.page) return;
+  if (plain) {
+    if (!in || !ts.page) return;
     uint8_t* dst = ts.page + d.off0 + ts.slot * d.pitch;
     if (p.fmt == STARKV_FMT_F32)
       reinterpret_cast<float*>(dst)[i] = c;
@@ -100,12 +104,8 @@ __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ Stor
     return;
   }
   __half* sc = ts.page ? reinterpret_cast<__half*>(ts.page + d.off2) + ts.slot * d.ng : nullptr;
-  if (cl < d.g8) {
+  if (is8) {
     // int8 group cl: channels [32 cl, min(32 cl + 32, n8))
-    const int i = cl * 32 + lane;
-    const bool in = i < d.n8;
-    const float c = in ? split_sum(src + i, p.split_stride, p.nsplit) : 0.f;
-    if (lout && in) lout[i] = c;
     const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
     const __half h = group_scale(amax, 127.f);
     const int q = quant_code(c, __half2float(h), 127);
@@ -114,11 +114,6 @@ __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ Stor
   } else {
     // int4 group gi: channels n8 + [32 gi, min(32 gi + 32, n4))
     const int gi = cl - d.g8;
-    const int n4 = d.rank - d.n8;
-    const int j = gi * 32 + lane;
-    const bool in = j < n4;
-    const float c = in ? split_sum(src + d.n8 + j, p.split_stride, p.nsplit) : 0.f;
-    if (lout && in) lout[d.n8 + j] = c;
     const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
     const __half h = group_scale(amax, 7.f);
     const int q = quant_code(c, __half2float(h), 7);
