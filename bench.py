@@ -242,8 +242,14 @@ def main():
             c()
     torch.cuda.synchronize(dev)
     assert lc.status.item() == 0, f"device status {lc.status.item()}"
-    # the step's launches replay from CUDA graphs (same kernels, same arguments), so the
-    # timed loop is not bound by host-side argument checks and launch latency
+    # The step's launches replay from CUDA graphs (same kernels, same arguments), so the timed
+    # loops are not bound by host-side argument checks and launch latency.  One graph holds
+    # the whole step (append, partials, combine: its kernels start with programmatic
+    # dependent launch); per-phase graphs time the split kernel on its own.
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph):
+        for c in calls:
+            c()
     graphs = []
     for c in calls:
         g_ = torch.cuda.CUDAGraph()
@@ -252,28 +258,35 @@ def main():
         graphs.append(g_)
     for _ in range(3):
         flush.fill_(1)
+        step_graph.replay()
+        flush.fill_(1)
         for g_ in graphs:
             g_.replay()
     torch.cuda.synchronize(dev)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
+        # (1) whole steps: the throughput
         for i in range(args.steps):
             flush.fill_(i & 0xFF)  # 256 MiB write: L2 holds nothing of the previous step
-            e = evs[i]
-            e[0].record(stream)
+            evs[i][0].record(stream)
+            step_graph.replay()
+            evs[i][1].record(stream)
+        # (2) the split kernel alone, between the same append and combine
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
             graphs[0].replay()
-            e[1].record(stream)
+            sevs[i][0].record(stream)
             graphs[1].replay()
-            e[2].record(stream)
+            sevs[i][1].record(stream)
             graphs[2].replay()
-            e[3].record(stream)
         torch.cuda.synchronize(dev)
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    split_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    split_ms = [e[0].elapsed_time(e[1]) for e in sevs]
     if world > 1:
         dist.barrier()
     # device time of the K steps, max over ranks; every rank processed B sequences

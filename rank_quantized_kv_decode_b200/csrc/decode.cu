@@ -414,6 +414,8 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   else
     __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tmem = misc[0];
   // the pair's MMA-side barriers live in the leader CTA
   auto leader_bar = [&](int i) { return CG == 2 ? mapa_shared(bar(i), 0) : bar(i); };
@@ -1054,6 +1056,8 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
 // One CTA per (sequence, query head): merge the tile partials (m in log2 units, l, a[r]),
 // normalise, then o = a B_v,g.
 __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int bh = blockIdx.x;
   const int b = bh / p.H, h = bh % p.H, g = h / p.G;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1153,13 +1157,15 @@ static cudaError_t launch_one(const DecodeParams& p, const CUtensorMap& tmA,
   cfg.blockDim = dim3(Fmt<FMT>::kWarps * 32, 1, 1);
   cfg.dynamicSmemBytes = p.smem_bytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (CG > 1) {
     // a persistent grid must be co-resident: not every SM can host half of a CTA pair
     // (pairs stay inside a GPC), so cap the grid at the pairs that fit at once
@@ -1217,8 +1223,7 @@ cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
 }
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t s) {
-  decode_combine_kernel<<<p.batch * p.H, 128, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(decode_combine_kernel, dim3(p.batch * p.H), dim3(128), 0, s, p);
 }
 
 size_t decode_smem_limit() { return 232448; }

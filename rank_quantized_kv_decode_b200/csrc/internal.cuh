@@ -1,6 +1,7 @@
 // Device-side parameter blocks and launch entry points shared by the kernels and the C ABI.
 #pragma once
 #include <string>
+#include <utility>
 
 #include "ptx.cuh"
 
@@ -79,6 +80,24 @@ struct DecodeParams {
 void set_error_message(const std::string& msg);
 
 // Launchers (defined in the .cu files; return cudaError_t of the launch).
+// Launch with programmatic stream serialization: the kernel may be scheduled while the one
+// before it on the stream finishes; it calls pdl_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_store(const StoreParams& p, cudaStream_t s);
 cudaError_t launch_dequant(const StoreParams& p, cudaStream_t s);
 cudaError_t launch_rope_init(float2* table, int half_dim, int rows_fine, int tiles, double theta,

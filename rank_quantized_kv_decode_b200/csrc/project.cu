@@ -62,6 +62,8 @@ __global__ void __launch_bounds__(ProjFmt<FMT>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tmem = misc[0];
   WaitCtl wc{reinterpret_cast<volatile int*>(misc + 1), p.status, p.timeout_ns};
 
@@ -188,14 +190,15 @@ cudaError_t launch_project(int fmt, const ProjParams& p, const CUtensorMap& tmX,
     e = cudaFuncSetAttribute(project_kernel<STARKV_FMT_F32>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    project_kernel<STARKV_FMT_F32><<<grid, ProjFmt<STARKV_FMT_F32>::kThreads, smem, s>>>(p, tmX, tmA);
+    e = launch_pdl(project_kernel<STARKV_FMT_F32>, grid, dim3(ProjFmt<STARKV_FMT_F32>::kThreads),
+                   smem, s, p, tmX, tmA);
   } else {
     e = cudaFuncSetAttribute(project_kernel<STARKV_FMT_BF16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    project_kernel<STARKV_FMT_BF16><<<grid, 192, smem, s>>>(p, tmX, tmA);
+    e = launch_pdl(project_kernel<STARKV_FMT_BF16>, grid, dim3(192), smem, s, p, tmX, tmA);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace starkv

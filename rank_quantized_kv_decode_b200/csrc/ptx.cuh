@@ -41,6 +41,17 @@ __device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
                : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization
+// may start while the kernel before it on the stream is still running: it does its setup
+// (barriers, TMEM, tensor-map prefetch), then waits here until that kernel has completed and
+// its memory is visible, and only then touches global memory.  Because every kernel of the
+// path waits before it completes, kernels still complete in stream order.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// let the next kernel on the stream be scheduled (its own pdl_wait still orders its reads)
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

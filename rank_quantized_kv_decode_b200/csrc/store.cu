@@ -71,6 +71,8 @@ __device__ __forceinline__ float split_sum(const float* src, long long stride, i
 // One warp per (token, latent, 32-channel chunk): lane = channel.  In the int8/int4 format a
 // chunk is one quantisation group (the int8 groups, then the int4 groups of the latent).
 __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ StoreParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= p.n_tok * p.chunks_per_token) return;  // whole warp
@@ -180,8 +182,7 @@ __global__ void rope_init_kernel(float2* table, int half_dim, int rows, double t
 cudaError_t launch_store(const StoreParams& p, cudaStream_t s) {
   const long long warps = (long long)p.n_tok * p.chunks_per_token;
   if (warps == 0) return cudaSuccess;
-  store_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(store_kernel, dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, s, p);
 }
 
 cudaError_t launch_dequant(const StoreParams& p, cudaStream_t s) {
