@@ -220,7 +220,7 @@ constexpr uint32_t kNoRow = 0xFFFFFFFFu;
 
 template <bool SMEM, class BaseFn>
 __device__ __forceinline__ void dequant_rows8(uint32_t dst, const LatDesc& kd, int k0, int ch,
-                                              int row0, BaseFn key_base) {
+                                              int row0, BaseFn key_base, uint32_t safe = 0) {
   const bool i8 = k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0;
   const bool i4 = !i8 && k0 >= kd.n8 && ((k0 - kd.n8) & 7) == 0 && k0 + 8 <= kd.rank &&
                   (kd.nb4 & 3) == 0;
@@ -240,17 +240,20 @@ __device__ __forceinline__ void dequant_rows8(uint32_t dst, const LatDesc& kd, i
       cy[it] = 0u;
       sb[it] = 0;
       if constexpr (SMEM) {
-        if (b != kNoRow) {
-          const uint32_t a = b + coff + prow * cpitch;
-          if (i8) {
-            const uint2 raw = ld_shared_v2(a);
-            cx[it] = raw.x;
-            cy[it] = raw.y;
-          } else {
-            cx[it] = ld_shared_u32(a);
-          }
-          sb[it] = ld_shared_u16(b + soff + prow * 2 * kd.ng);
+        // branch-free (a missing row reads the readable address ``safe`` and gets scale 0):
+        // loads under a branch per row were not batched and cost 2.3x here
+        const bool ok = b != kNoRow;
+        const uint32_t bs = ok ? b : safe;
+        const uint32_t a = bs + coff + prow * cpitch;
+        if (i8) {
+          const uint2 raw = ld_shared_v2(a);
+          cx[it] = raw.x;
+          cy[it] = raw.y;
+        } else {
+          cx[it] = ld_shared_u32(a);
         }
+        const unsigned short sv = ld_shared_u16(bs + soff + prow * 2 * kd.ng);
+        sb[it] = ok ? sv : static_cast<unsigned short>(0);
       } else {
         if (b) {
           if (i8) {
@@ -960,7 +963,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           dequant_rows8<true>(smem_u32(sA + kb * kAStage), kd, kb * 64 + ch * 8, ch, tid >> 3,
                               [&](int it, int r) -> uint32_t {
                                 return r < U.nvalid ? (it < 4 ? pb0 : pb1) : kNoRow;
-                              });
+                              }, codes);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -1009,7 +1012,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
               dequant_rows8<true>(dst, kd, kb * 64 + ch * 8, ch, tid >> 3,
                                   [&](int it, int r) -> uint32_t {
                                     return r < U.nvalid ? (it < 4 ? pb0 : pb1) : kNoRow;
-                                  });
+                                  }, codes);
             } else {
               const uint8_t* gb0 = U.page0 >= 0 ? p.cache + (long long)U.page0 * p.page_bytes : nullptr;
               const uint8_t* gb1 = U.page1 >= 0 ? p.cache + (long long)U.page1 * p.page_bytes : nullptr;
