@@ -326,8 +326,9 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
   constexpr int HALF = HD / 2;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base (SW128 tiles), by pointer arithmetic on the shared array so that the
+  // compiler keeps the address space and emits shared-memory instructions for every access
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   static_assert(CG == 1 || !Fmt<FMT>::kSplit, "fp32 latents use single-CTA tiles");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.stages, NVB = p.nvb;

@@ -30,8 +30,9 @@ __global__ void __launch_bounds__(ProjFmt<FMT>::kThreads, 1)
   constexpr uint32_t kAStride = kSplit ? 2 * kAStage : kAStage;
   constexpr uint32_t kBStride = kSplit ? 2 * kBStage : kBStage;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base (SW128 tiles), by pointer arithmetic on the shared array so that the
+  // compiler keeps the address space and emits shared-memory instructions for every access
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int S = p.stages;
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * kAStride;
