@@ -30,7 +30,7 @@ MEASURED_PEAKS = os.path.join(HERE, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram bytes per launch of the split kernel from the committed ncu capture of this workload
 # (profiles/decode_split_bf16_llama2_b8_ctx4096.md); set to None when the kernel changes
-SPLIT_TRAFFIC_BYTES = None  # recaptured after each change of the kernel
+SPLIT_TRAFFIC_BYTES = 149060864  # 142.961664 MB read + 6.099200 MB written
 
 THROTTLE_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                  0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
@@ -345,6 +345,9 @@ def main():
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tc, "unit": "TFLOP/s",
                      "frac": tflops / peak_tc, "traffic": SPLIT_TRAFFIC_BYTES,
                      "peak_source": f"{src} bf16 burst", "kernel": "decode_split_kernel",
+                     "peak_sustained": pk.get("bf16_tflops_sustained"),
+                     "frac_of_sustained": (tflops / pk["bf16_tflops_sustained"]
+                                           if pk.get("bf16_tflops_sustained") else None),
                      "flop_per_launch": recon_flop, "split_ms": split_s * 1000.0,
                      "hbm_achieved_gbs": hbm_gbs, "hbm_peak_gbs": pk["hbm_gbs"],
                      "hbm_frac": hbm_gbs / pk["hbm_gbs"], "hbm_bytes_per_launch": bytes_alg},
