@@ -353,7 +353,8 @@ def main():
                      "hbm_frac": hbm_gbs / pk["hbm_gbs"], "hbm_bytes_per_launch": bytes_alg},
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        # pass 1: append (projection + store), split, combine per step; pass 2: the same
+        "gpu_launches": 8 * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
