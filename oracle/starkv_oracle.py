@@ -417,15 +417,15 @@ def reconstruct_keys(C_k: np.ndarray, B_k: np.ndarray) -> np.ndarray:
     return np.asarray(C_k, np.float64) @ np.asarray(B_k, np.float64)
 
 
-def decode_attention(q, C_k, C_v, B_k, B_v, theta: float, n_kv_heads: int, heads=None):
-    """Single-token decode attention of one sequence from its stored latents.
+def latent_attention(q, C_k, C_v, B_k, theta: float, n_kv_heads: int, heads=None):
+    """Single-token decode attention of one sequence in the latent space of the values.
 
     q   : (H, d) query of the token at position L-1, before RoPE.
     C_k : (L, r_k) key latents;  C_v: list over KV heads g of (L, r_g) value latents.
-    B_k : (r_k, H_kv*d);  B_v: list over g of (r_g, d).
+    B_k : (r_k, H_kv*d).
     Steps: K = C_k B_k; per head g(h) = h // (H/H_kv): RoPE on K_g at positions 0..L-1 and
-    on q_h at L-1; scores q'.k'/sqrt(d); softmax (max subtracted, fp64); a = p C_v,g;
-    o_h = a B_v,g.  Returns (H, d), or only ``heads`` rows (in that order) when given."""
+    on q_h at L-1; scores q'.k'/sqrt(d); softmax (max subtracted, fp64); a_h = p C_v,g.
+    Returns the list of a_h (each (r_g(h),)) for ``heads`` (default: all, in order)."""
     q = np.asarray(q, dtype=np.float64)
     H, d = q.shape
     G = H // n_kv_heads
@@ -445,9 +445,39 @@ def decode_attention(q, C_k, C_v, B_k, B_v, theta: float, n_kv_heads: int, heads
         s = s - s.max()
         p = np.exp(s)
         p = p / p.sum()
-        a = p @ np.asarray(C_v[g], np.float64)
-        out.append(a @ np.asarray(B_v[g], np.float64))
-    return np.array(out)
+        out.append(p @ np.asarray(C_v[g], np.float64))
+    return out
+
+
+def decode_attention(q, C_k, C_v, B_k, B_v, theta: float, n_kv_heads: int, heads=None):
+    """Single-token decode attention of one sequence from its stored latents: the latent
+    outputs a_h of latent_attention, up-projected o_h = a_h B_v,g(h) (B_v: list over g of
+    (r_g, d)).  Returns (H, d), or only ``heads`` rows (in that order) when given."""
+    H = np.asarray(q).shape[0]
+    G = H // n_kv_heads
+    heads = list(range(H)) if heads is None else list(heads)
+    a = latent_attention(q, C_k, C_v, B_k, theta, n_kv_heads, heads)
+    return np.array([a_h @ np.asarray(B_v[h // G], np.float64) for a_h, h in zip(a, heads)])
+
+
+def absorb_output_weights(B_v, W_o, n_q_heads: int) -> list:
+    """Weight absorption (STAR-KV technical summary, Methodology §2: the value up-projection
+    is folded into the attention output projection, so values are never reconstructed): for
+    each query head h, M_h = B_v,g(h) W_o,h with W_o,h the rows [h d, (h+1) d) of W_o
+    (H d x d_out).  Returns the list of M_h, each (r_g(h), d_out)."""
+    W_o = np.asarray(W_o, np.float64)
+    n_kv = len(B_v)
+    G = n_q_heads // n_kv
+    d = np.asarray(B_v[0]).shape[1]
+    return [np.asarray(B_v[h // G], np.float64) @ W_o[h * d:(h + 1) * d] for h in range(n_q_heads)]
+
+
+def decode_attention_absorbed(q, C_k, C_v, B_k, M, theta: float, n_kv_heads: int) -> np.ndarray:
+    """The attention block's output for the decoded token with absorbed weights:
+    y = sum_h a_h M_h (a_h from latent_attention, M_h from absorb_output_weights), i.e.
+    (concat_h o_h) W_o without forming o.  Returns (d_out,)."""
+    a = latent_attention(q, C_k, C_v, B_k, theta, n_kv_heads)
+    return np.sum([a_h @ M_h for a_h, M_h in zip(a, M)], axis=0)
 
 
 def project(x, A) -> np.ndarray:
