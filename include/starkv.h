@@ -235,6 +235,39 @@ STARKV_API starkv_status starkv_decode_combine(const starkv_layout* lay, const i
                                                const void* workspace, size_t workspace_bytes,
                                                float* out, starkv_stream_t stream);
 
+/* Weight absorption (STAR-KV technical summary, Methodology §2: the values' up-projection is
+ * folded into the attention output projection, so values are never reconstructed).  With one
+ * value latent per KV head, query head h gets M_h = B_v,g(h) W_o,h, where W_o,h is the rows
+ * [h*d, (h+1)*d) of the output projection W_o (n_q_heads*d x d_out), and the attention block's
+ * output for the decoded token of sequence b is y_b = sum_h a_b,h M_h, a_b,h the normalised
+ * latent-space output of head h.
+ *
+ * starkv_absorbed_sizes: rows of M (sum over query heads of r_g(h)) and the bytes of scratch
+ * that starkv_decode_combine_absorbed needs for ``batch`` sequences.  Host only. */
+STARKV_API starkv_status starkv_absorbed_sizes(const starkv_layout* lay, int32_t batch,
+                                               int32_t d_out, int64_t* m_rows,
+                                               size_t* scratch_bytes);
+
+/* Build M once (setup, fp32):
+ *   Bv  device fp32 [value_rank_total][d], as for starkv_decode_attention
+ *   Wo  device fp32 [n_q_heads*d][d_out], row-major (o_concat . Wo)
+ *   M   device fp32 [m_rows][d_out]: the r_g rows of query head h start at
+ *       G * (sum of r_g' over KV heads g' < g) + (h mod G) * r_g. */
+STARKV_API starkv_status starkv_absorb_output_weights(const starkv_layout* lay, const float* Bv,
+                                                      const float* Wo, int32_t d_out, float* M,
+                                                      starkv_stream_t stream);
+
+/* The combine step with absorbed weights: merge the partial records of every (b, h) as
+ * starkv_decode_combine does, keep a_b,h, then out[b][:] = sum_h a_b,h M_h.
+ *   M        from starkv_absorb_output_weights for the same d_out
+ *   scratch  device, >= scratch_bytes of starkv_absorbed_sizes, 16-byte aligned
+ *   out      device fp32 [batch][d_out]; seq_len 0 gives a zero row
+ * Other arguments as starkv_decode_combine. */
+STARKV_API starkv_status starkv_decode_combine_absorbed(
+    const starkv_layout* lay, const int32_t* seq_lens, int32_t batch, int32_t max_pages,
+    const float* M, int32_t d_out, const void* workspace, size_t workspace_bytes, void* scratch,
+    size_t scratch_bytes, float* out, starkv_stream_t stream);
+
 /* starkv_decode_attention without a workspace argument, for callers that cannot allocate
  * device memory: a plugin inside a host process whose memory pool has already reserved the
  * GPU's memory, a C caller with no device allocator, or a loop where a cudaMalloc is not

@@ -67,6 +67,11 @@ EXPORTS = {
     "starkv_decode_attention_noalloc": (i32, [ctypes.POINTER(Layout), vp, vp, i64, vp, i32, vp, i32,
                                               vp, vp, vp, sz, vp, ctypes.POINTER(DecodeOpts), vp,
                                               vp]),
+    "starkv_absorbed_sizes": (i32, [ctypes.POINTER(Layout), i32, i32, ctypes.POINTER(i64),
+                                    ctypes.POINTER(sz)]),
+    "starkv_absorb_output_weights": (i32, [ctypes.POINTER(Layout), vp, vp, i32, vp, vp]),
+    "starkv_decode_combine_absorbed": (i32, [ctypes.POINTER(Layout), vp, i32, i32, vp, i32, vp, sz,
+                                             vp, sz, vp, vp]),
     "starkv_diag_bounded_wait": (i32, [i32, vp, vp]),
     "starkv_last_error": (ctypes.c_char_p, []),
     "starkv_version": (i32, []),

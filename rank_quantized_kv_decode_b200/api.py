@@ -137,6 +137,31 @@ def decode_combine(lay, seq_lens, max_pages: int, Bv, workspace, out, stream=Non
         _stream(stream)), "starkv_decode_combine")
 
 
+def absorbed_sizes(lay, batch: int, d_out: int) -> tuple[int, int]:
+    """(rows of the absorbed matrix M, scratch bytes of decode_combine_absorbed)."""
+    rows, nbytes = ctypes.c_int64(0), ctypes.c_size_t(0)
+    L.check(L.load().starkv_absorbed_sizes(ctypes.byref(lay), batch, d_out, ctypes.byref(rows),
+                                           ctypes.byref(nbytes)), "starkv_absorbed_sizes")
+    return int(rows.value), int(nbytes.value)
+
+
+def absorb_output_weights(lay, Bv, Wo, M, stream=None) -> None:
+    """M[rows of head h] = B_v,g(h) Wo[h d:(h+1) d] (fp32, on the device)."""
+    L.check(L.load().starkv_absorb_output_weights(ctypes.byref(lay), _ptr(Bv), _ptr(Wo),
+                                                  Wo.shape[1], _ptr(M), _stream(stream)),
+            "starkv_absorb_output_weights")
+
+
+def decode_combine_absorbed(lay, seq_lens, max_pages: int, M, workspace, scratch, out,
+                            stream=None) -> None:
+    """Merge the partial records and write out[b] = sum_h a_b,h M_h (out: [batch][d_out])."""
+    L.check(L.load().starkv_decode_combine_absorbed(
+        ctypes.byref(lay), _ptr(seq_lens), seq_lens.shape[0], max_pages, _ptr(M), out.shape[1],
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(scratch),
+        scratch.numel() * scratch.element_size(), _ptr(out), _stream(stream)),
+        "starkv_decode_combine_absorbed")
+
+
 def diag_bounded_wait(timeout_ms: int, status, stream=None) -> None:
     L.check(L.load().starkv_diag_bounded_wait(timeout_ms, _ptr(status), _stream(stream)),
             "starkv_diag_bounded_wait")

@@ -710,6 +710,106 @@ starkv_status starkv_decode_attention(const starkv_layout* lay, const void* q, c
   return STARKV_OK;
 }
 
+// ---------------------------------------------------------------- weight absorption
+static void fill_absorb(const starkv_layout* lay, int32_t d_out, int32_t batch, AbsorbParams& a) {
+  std::memset(&a, 0, sizeof(a));
+  const starkv_config& c = lay->cfg;
+  a.H = c.n_q_heads;
+  a.G = c.n_q_heads / c.n_kv_heads;
+  a.d = c.head_dim;
+  a.d_out = d_out;
+  a.key_rank_cols = c.key_rank;
+  int rv = 0;
+  for (int g = 0; g < c.n_kv_heads; ++g) {
+    a.vh[g] = lat_desc(lay->seg[1 + g]);
+    rv += lay->seg[1 + g].rank;
+  }
+  a.m_rows = a.G * rv;
+  // splits of M's rows (32 rows at least): with the column tiles and the 8-sequence groups,
+  // enough CTAs for the HBM stream of M
+  a.ksplit = std::max(1, std::min(32, a.m_rows / 32));
+  a.krows = ceil_div(a.m_rows, a.ksplit);
+  a.ksplit = ceil_div(a.m_rows, a.krows);
+}
+
+starkv_status starkv_absorbed_sizes(const starkv_layout* lay, int32_t batch, int32_t d_out,
+                                    int64_t* m_rows, size_t* scratch_bytes) {
+  starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  if (batch < 0 || d_out < 1 || d_out > (1 << 20))
+    return fail(STARKV_ERR_INVALID_ARG, "batch < 0 or d_out outside [1, 2^20]");
+  if (!m_rows || !scratch_bytes) return fail(STARKV_ERR_INVALID_ARG, "NULL output pointer");
+  AbsorbParams a;
+  fill_absorb(lay, d_out, batch, a);
+  *m_rows = a.m_rows;
+  const size_t rows_a = static_cast<size_t>(batch) * a.m_rows;
+  *scratch_bytes = (rows_a + 63) / 64 * 64 * sizeof(float) +
+                   static_cast<size_t>(a.ksplit) * batch * d_out * sizeof(float);
+  return STARKV_OK;
+}
+
+starkv_status starkv_absorb_output_weights(const starkv_layout* lay, const float* Bv,
+                                           const float* Wo, int32_t d_out, float* M,
+                                           starkv_stream_t stream) {
+  starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  if (d_out < 1 || d_out > (1 << 20)) return fail(STARKV_ERR_INVALID_ARG, "d_out outside [1, 2^20]");
+  if (!Bv || !Wo || !M) return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
+  DevInfo info;
+  st = current_device(info);
+  if (st != STARKV_OK) return st;
+  AbsorbParams a;
+  fill_absorb(lay, d_out, 1, a);
+  a.Bv = Bv;
+  a.Wo = Wo;
+  a.M = M;
+  cudaError_t e = launch_absorb_weights(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "weight absorption launch");
+  return STARKV_OK;
+}
+
+starkv_status starkv_decode_combine_absorbed(const starkv_layout* lay, const int32_t* seq_lens,
+                                             int32_t batch, int32_t max_pages, const float* M,
+                                             int32_t d_out, const void* workspace,
+                                             size_t workspace_bytes, void* scratch,
+                                             size_t scratch_bytes, float* out,
+                                             starkv_stream_t stream) {
+  int64_t m_rows = 0;
+  size_t need = 0;
+  starkv_status st = starkv_absorbed_sizes(lay, batch, d_out, &m_rows, &need);
+  if (st != STARKV_OK) return st;
+  if (batch == 0) return STARKV_OK;
+  if (!M || !scratch || !out) return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
+  if (scratch_bytes < need) return fail(STARKV_ERR_WORKSPACE, "absorbed-output scratch too small");
+  if (reinterpret_cast<uintptr_t>(scratch) & 15)
+    return fail(STARKV_ERR_INVALID_ARG, "scratch must be 16-byte aligned");
+  DecodeParams p;
+  CUtensorMap tmA, tmB;
+  int grid = 0;
+  // the merge of the partial records: the combine without its up-projection (M stands in
+  // for B_v in the argument checks and is not read by it)
+  st = plan_decode(lay, nullptr, nullptr, 0, nullptr, max_pages, seq_lens, batch, nullptr, M,
+                   nullptr, 0, out, const_cast<void*>(workspace), workspace_bytes, nullptr,
+                   nullptr, false, true, p, tmA, tmB, grid);
+  if (st != STARKV_OK) return st;
+  float* A = reinterpret_cast<float*>(scratch);
+  p.a_out = A;
+  p.a_stride = static_cast<int>(m_rows);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_combine(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode merge launch");
+  AbsorbParams a;
+  fill_absorb(lay, d_out, batch, a);
+  a.M = const_cast<float*>(M);  // read only by the product kernels
+  a.A = A;
+  a.part = A + (static_cast<size_t>(batch) * m_rows + 63) / 64 * 64;
+  a.y = out;
+  a.batch = batch;
+  e = launch_absorbed_output(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "absorbed output launch");
+  return STARKV_OK;
+}
+
 starkv_status starkv_diag_bounded_wait(int32_t timeout_ms, int32_t* dev_status,
                                       starkv_stream_t stream) {
   if (timeout_ms < 1 || timeout_ms > 10000)

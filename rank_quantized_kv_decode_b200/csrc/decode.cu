@@ -1073,8 +1073,17 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   float* outp = p.out + ((long long)b * p.H + h) * p.d;
   int L = p.seq_lens[b];
   L = max(0, min(L, p.max_pages * kPage));
+  // merge mode: the normalised a_h goes to its rows in a_out (query heads of KV head g
+  // are consecutive blocks of r_g rows after the rows of the heads of KV heads < g)
+  float* a_row = p.a_out ? p.a_out + (long long)b * p.a_stride + p.G * (vd.col - p.key_rank_cols) +
+                               (h % p.G) * r
+                         : nullptr;
   if (L == 0) {
-    for (int c = tid; c < p.d; c += 128) outp[c] = 0.f;
+    if (a_row) {
+      for (int i = tid; i < r; i += 128) a_row[i] = 0.f;
+    } else {
+      for (int c = tid; c < p.d; c += 128) outp[c] = 0.f;
+    }
     return;
   }
   const int T = (L + kTile - 1) / kTile;
@@ -1129,6 +1138,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   const float l = s_acc[0][128] + s_acc[1][128] + s_acc[2][128] + s_acc[3][128];
   const float inv = l > 0.f ? 1.f / l : 0.f;
   s_a[tid] = tid < r ? (s_acc[0][tid] + s_acc[1][tid] + s_acc[2][tid] + s_acc[3][tid]) * inv : 0.f;
+  if (a_row) {
+    if (tid < r) a_row[tid] = s_a[tid];
+    return;
+  }
   __syncthreads();
   // o_c = sum_i a_i B_v[i][c], 32 rows of B_v in flight at a time (a_i = 0 for i >= r)
   const float* Bv = p.Bv + (long long)(vd.col - p.key_rank_cols) * p.d;

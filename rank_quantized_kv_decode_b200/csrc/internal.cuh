@@ -58,6 +58,8 @@ struct DecodeParams {
   float* ws;          // partial records
   int tiles_max, rec; // tiles per sequence slot, floats per record
   float* out;         // [batch][H][d]
+  float* a_out;       // when set, the combine writes the normalised latent outputs a_h here
+  int a_stride;       // floats per sequence row of a_out (rows of all query heads)
   int* status;
   unsigned long long timeout_ns;
   int H, Hkv, G, d, rk, key_rank_cols;
@@ -99,6 +101,20 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 cudaError_t launch_store(const StoreParams& p, cudaStream_t s);
+
+// Weight absorption (attention output projection folded into the value up-projection).
+struct AbsorbParams {
+  const float* Bv;  // [R_v][d]
+  const float* Wo;  // [H * d][d_out]
+  float* M;         // [m_rows][d_out]: rows of query head h at row_start(h)
+  const float* A;   // [batch][m_rows] latent outputs a_h (normalised)
+  float* part;      // [ksplit][batch][d_out]
+  float* y;         // [batch][d_out]
+  int H, G, d, d_out, m_rows, batch, ksplit, krows, key_rank_cols;
+  LatDesc vh[STARKV_MAX_KV_HEADS];
+};
+cudaError_t launch_absorb_weights(const AbsorbParams& p, cudaStream_t s);
+cudaError_t launch_absorbed_output(const AbsorbParams& p, cudaStream_t s);
 cudaError_t launch_dequant(const StoreParams& p, cudaStream_t s);
 cudaError_t launch_rope_init(float2* table, int half_dim, int rows_fine, int tiles, double theta,
                              int head_dim, cudaStream_t s);

@@ -87,6 +87,18 @@ def test_alloc_sizes(lib):
     assert s.append_workspace_bytes >= 8192 * lay.proj_cols * 4
 
 
+def test_absorbed_sizes(lib):
+    rv = [8, 48, 37, 17, 32, 29, 40, 45]
+    lay = api.layout_init(api.make_config(32, 8, 128, 4096, 256, rv, "mixed", 500000.0))
+    rows, nbytes = api.absorbed_sizes(lay, 3, 4096)
+    # four query heads per KV head, each with the r_g rows of its group
+    assert rows == 4 * sum(rv)
+    # the latent outputs of every (sequence, head), then at least one split of [3][4096] partials
+    assert nbytes >= 3 * rows * 4 + 3 * 4096 * 4
+    with pytest.raises(L.StarkvError):
+        api.absorbed_sizes(lay, 3, 0)
+
+
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 96, L.ERR_UNSUPPORTED),
     ("n_kv_heads", 0, L.ERR_INVALID_ARG),
