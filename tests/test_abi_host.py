@@ -99,6 +99,14 @@ def test_absorbed_sizes(lib):
         api.absorbed_sizes(lay, 3, 0)
 
 
+def test_absorbed_combine_rejects_small_scratch_before_touching_the_device(lib):
+    lay = api.layout_init(api.make_config(32, 8, 128, 4096, 256, [32] * 8, "mixed", 500000.0))
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
+    st = lib.starkv_decode_combine_absorbed(ctypes.byref(lay), fake, 2, 4, fake, 64, fake, 1 << 30,
+                                            fake, 16, fake, None)
+    assert st == L.ERR_WORKSPACE
+
+
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 96, L.ERR_UNSUPPORTED),
     ("n_kv_heads", 0, L.ERR_INVALID_ARG),
