@@ -93,14 +93,18 @@ struct WaitCtl {
   uint64_t timeout_ns;
 };
 
-static __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& w) {
+// The control block's fields travel by value (registers): taking the block by reference made
+// the caller keep it in local memory and reload it on every slow wait.
+static __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity,
+                                              volatile int* abort_flag, int* status,
+                                              uint64_t timeout_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*w.abort_flag) return false;
-    if ((it & 7u) == 0u && globaltimer_ns() - t0 > w.timeout_ns) {
-      *w.abort_flag = 1;
-      if (w.status) atomicOr(w.status, STARKV_DEV_TIMEOUT);
+    if (*abort_flag) return false;
+    if ((it & 7u) == 0u && globaltimer_ns() - t0 > timeout_ns) {
+      *abort_flag = 1;
+      if (status) atomicOr(status, STARKV_DEV_TIMEOUT);
       return false;
     }
   }
@@ -108,7 +112,7 @@ static __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, con
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const WaitCtl& w) {
   if (mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, w);
+  return wait_slow(bar, parity, w.abort_flag, w.status, w.timeout_ns);
 }
 
 // Named barrier over a subset of warps (id 1..15; id 0 is __syncthreads).
