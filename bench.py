@@ -30,7 +30,7 @@ MEASURED_PEAKS = os.path.join(HERE, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram bytes per launch of the split kernel from the committed ncu capture of this workload
 # (profiles/decode_split_bf16_llama2_b8_ctx4096.md); set to None when the kernel changes
-SPLIT_TRAFFIC_BYTES = None  # recaptured after each change of the kernel
+SPLIT_TRAFFIC_BYTES = 146703104  # 143.034112 MB read + 3.668992 MB written
 
 THROTTLE_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                  0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
