@@ -1,23 +1,28 @@
 // Decode attention read straight from the latent cache (sm_100a).
 //
-// Split kernel (persistent, warp-specialised, one CTA per SM).  A work unit is one
-// 128-token tile (two 64-token pages) of one sequence and a range of 256-column chunks of
-// the reconstructed keys (2 KV heads of d=128, or 4 of d=64):
+// Split kernel (persistent, warp-specialised, one CTA per SM, or a CTA pair per cluster with
+// cta_group::2).  A work unit is one 128-token tile (two 64-token pages) of one sequence --
+// 256 tokens for a pair, each CTA owning 128 -- and a range of 256-column chunks of the
+// reconstructed keys (2 KV heads of d=128, or 4 of d=64):
 //   warp 0      TMA producer: latent k-blocks of the two pages (f32/bf16) and B_k^T k-blocks
 //   warp 1      tcgen05 issuer: K_chunk = C_k(128 x r_k) * B_k(r_k x 256) into TMEM (fp32),
-//               double-buffered accumulators (2 x 256 columns)
+//               double-buffered accumulators (2 x 256 columns); M = 256 across a pair
 //   warp 2      bulk-copy producer of the value latents of the chunk's heads (both pages)
-//   warps 4-11  two epilogue warpgroups, one per 128 TMEM columns: thread = token row;
-//               RoPE on the key row, scores against the rotated queries of the GQA group,
-//               tile-local softmax (max, sum), latent P.C_v, one partial per query head
-//   warps 12-15 (int8/int4 format) dequantisers: codes * fp16 scale -> fp16 operand tile in
-//               the 128-byte-swizzled layout the tensor core reads
+//   warp 3      int8/int4 keys: bulk-copy stager of the tile's key codes
+//   warps 4-11  two epilogue warpgroups, thread = token row (TMEM lane): warpgroup w rotates
+//               and dots half of the RoPE pairs of every head of the chunk; then, for the
+//               heads it owns, the tile-local softmax (max, sum) and the latent P.C_v, one
+//               partial record per query head
+//   warps 12-15 int8/int4 keys: dequantisers (codes * fp16 scale -> fp16 operand tile in the
+//               128-byte-swizzled layout the tensor core reads), once per tile into resident
+//               slots (rank <= 256) or per ring stage; fp32 latents: tf32 hi/lo splitters
 // The pages' point that joint key latents cost h x more to reconstruct (STAR-KV technical
 // summary, Methodology §2 "Hybrid Decomposition Strategy") is why the reconstruction runs
 // on the tensor cores: it is a dense (tokens x r_k) x (r_k x H_kv*d) contraction.
 //
 // Combine kernel: log-sum-exp merge of the per-tile partials of each (sequence, query head),
-// then the up-projection o_h = a_h B_v,g.
+// then the up-projection o_h = a_h B_v,g -- or, for the absorbed output, the normalised a_h
+// alone.
 #include "internal.cuh"
 
 namespace starkv {
