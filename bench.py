@@ -111,6 +111,7 @@ class OracleDecode:
         self.ref = ref = ref_for(workload_index, False)
         self.w = ref.w
         self.q = ref.queries()
+        n_seq = max(1, min(n_seq, self.w["batch"]))  # the workload may hold fewer sequences
         self.seqs = [ref.stored(ref.sequence_latents(b)) for b in range(n_seq)]
         self.cores = (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
                       else os.cpu_count())
