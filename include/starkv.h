@@ -18,12 +18,17 @@
  *   reconstruction overhead at inference; Methodology §2: JD costs h x more to reconstruct):
  *       K = C_k B_k, RoPE(K) per KV head, softmax(q' K'^T / sqrt(d)) per query head,
  *       a_h = p C_v,g(h), o_h = a_h B_v,g(h).
+ *   Optionally with the value up-projection folded into the output projection
+ *   (Methodology §2): y = sum_h a_h (B_v,g(h) W_o,h).
  *
  * Conventions shared by every entry point:
  *   - The caller owns all memory.  The library never allocates device memory, never
  *     synchronises and never frees.  Pointers marked "device" must be device pointers of
  *     the current device; pointers marked "host" are read before the call returns.
  *   - Every call is asynchronous on ``stream`` (a cudaStream_t; NULL = legacy default).
+ *     The kernels of append, decode and combine are launched with programmatic stream
+ *     serialisation: each may start its setup while the kernel before it on the stream
+ *     finishes, and waits for that kernel to complete before it touches global memory.
  *   - The return value reports argument validation and launch errors only.  Errors found
  *     on the device are OR-ed into ``*dev_status`` (device int32, zeroed by the caller),
  *     as STARKV_DEV_* bits, read by the caller after a synchronisation.
