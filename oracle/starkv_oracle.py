@@ -480,6 +480,40 @@ def decode_attention_absorbed(q, C_k, C_v, B_k, M, theta: float, n_kv_heads: int
     return np.sum([a_h @ M_h for a_h, M_h in zip(a, M)], axis=0)
 
 
+def decode_attention_hybrid(q, C_k, C_v, B_k, B_v, theta: float, n_kv_heads: int, heads=None):
+    """Decode attention with the pages' own assignment (STAR-KV technical summary,
+    Methodology §2 "Hybrid Decomposition Strategy": keys head-wise, values joint).
+
+    q   : (H, d) query of the token at position L-1, before RoPE.
+    C_k : list over KV heads g of (L, r_k,g) key latents;  B_k: list over g of (r_k,g, d).
+    C_v : (L, r_v) joint value latents;  B_v: (r_v, H_kv*d).
+    Steps: K_g = C_k,g B_k,g; RoPE on K_g at positions 0..L-1 and on q_h at L-1; scores
+    q'.k'/sqrt(d); softmax (max subtracted, fp64); a_h = p C_v in the joint latent space
+    (r_v values, the same space for every head); o_h = a_h B_v[:, g(h) d:(g(h)+1) d].
+    Returns (H, d), or only ``heads`` rows (in that order) when given."""
+    q = np.asarray(q, dtype=np.float64)
+    H, d = q.shape
+    G = H // n_kv_heads
+    L = np.asarray(C_v).shape[0]
+    heads = range(H) if heads is None else heads
+    pos = np.arange(L)
+    Cv = np.asarray(C_v, np.float64)
+    Bv = np.asarray(B_v, np.float64)
+    out = []
+    cache_k = {}
+    for h in heads:
+        g = h // G
+        if g not in cache_k:
+            cache_k[g] = apply_rope(np.asarray(C_k[g], np.float64) @ np.asarray(B_k[g], np.float64),
+                                    pos, theta)
+        s = cache_k[g] @ apply_rope(q[h], L - 1, theta) / math.sqrt(d)
+        s = s - s.max()
+        p = np.exp(s)
+        p = p / p.sum()
+        out.append((p @ Cv) @ Bv[:, g * d:(g + 1) * d])
+    return np.array(out)
+
+
 def project(x, A) -> np.ndarray:
     """Latent write of new tokens: c = x A, with A = [A_k | A_v,0 | A_v,1 | ...] [AB]."""
     return np.asarray(x, np.float64) @ np.asarray(A, np.float64)
