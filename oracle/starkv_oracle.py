@@ -36,6 +36,12 @@ Readings where the pages are silent (each is listed again in the design notes):
     the even channel.  int8 channels: the first ceil(r/4).
   * RoPE: half-split (rotate-half) form, theta_j = base^(-2j/d), 0-based positions, the
     decode query at position L-1.  Output fp32-comparable fp64.
+  * The pages' own quantiser [S3] (block-wise Hadamard, 4-bit outliers, 3-bit inliers):
+    outlier block = the leading ceil(r/5) channels; each block is rotated by normalised
+    Sylvester Hadamard matrices, one per set bit of its size (largest first), the transform
+    folded into the factors (A T, T^T B); then the quantiser above with 4 and 3 bits, groups
+    of 32 restarting at the block boundary; 3-bit codes packed eight to three bytes, code i
+    in bits [3i, 3i+3) of the little-endian 24-bit word, two's complement.
 """
 from __future__ import annotations
 
@@ -253,6 +259,119 @@ def quantize_latent(c, r: int):
     q8 = np.concatenate(q8) if q8 else np.zeros(0, np.int8)
     q4 = np.concatenate(q4) if q4 else np.zeros(0, np.int8)
     return q8, q4, np.array(scales, dtype=np.float16)
+
+
+# ======================================================================================
+# [S3] the pages' own format: block-wise Hadamard rotation, 4-bit / 3-bit
+# ======================================================================================
+def sylvester_hadamard(n: int) -> np.ndarray:
+    """Normalised Sylvester Hadamard matrix of order n (a power of two): entries +-1/sqrt(n),
+    H H^T = I."""
+    assert n >= 1 and n & (n - 1) == 0
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H / math.sqrt(n)
+
+
+def block_hadamard(n: int) -> np.ndarray:
+    """Orthogonal n x n transform for a block of n channels: normalised Sylvester blocks down
+    the diagonal, one per set bit of n, largest first."""
+    T = np.zeros((n, n))
+    at = 0
+    for k in reversed(range(max(n.bit_length(), 1))):
+        size = 1 << k
+        if n & size:
+            T[at:at + size, at:at + size] = sylvester_hadamard(size)
+            at += size
+    return T
+
+
+def hadamard_split(r: int) -> dict:
+    """Outlier block [0, n_hi) -- the leading fifth of the channels in singular-value order,
+    rounded up -- and inlier block [n_hi, r) [S3]."""
+    n_hi = -(-r // 5)
+    n_lo = r - n_hi
+    return dict(n_hi=n_hi, n_lo=n_lo, g_hi=-(-n_hi // GROUP), g_lo=-(-n_lo // GROUP))
+
+
+def hadamard_transform(r: int) -> np.ndarray:
+    """The block-wise transform of a rank-r latent: independent rotations of the outlier and
+    the inlier block [S3]."""
+    sp = hadamard_split(r)
+    T = np.zeros((r, r))
+    T[:sp["n_hi"], :sp["n_hi"]] = block_hadamard(sp["n_hi"])
+    T[sp["n_hi"]:, sp["n_hi"]:] = block_hadamard(sp["n_lo"])
+    return T
+
+
+def rotate_factors(A, B):
+    """Fold the transform into the factors ("zero overhead" [S3]): A' = A T, B' = T^T B, so
+    A' B' = A B and the latents x A' are the rotated latents."""
+    A = np.asarray(A, np.float64)
+    T = hadamard_transform(A.shape[1])
+    return A @ T, T.T @ np.asarray(B, np.float64)
+
+
+def quantize_hadamard_latent(c, r: int):
+    """One token's rotated rank-r latent (fp32) -> (4-bit codes of the outlier block, 3-bit
+    codes of the inlier block, fp16 scales [g_hi + g_lo]) [S3]."""
+    c = np.asarray(c, dtype=np.float32)
+    assert c.shape == (r,)
+    sp = hadamard_split(r)
+    n_hi, n_lo = sp["n_hi"], sp["n_lo"]
+    scales, qh, ql = [], [], []
+    for gi in range(sp["g_hi"]):
+        s, q = quantize_group(c[gi * GROUP:min((gi + 1) * GROUP, n_hi)], 4)
+        scales.append(s)
+        qh.append(q)
+    for gi in range(sp["g_lo"]):
+        s, q = quantize_group(c[n_hi + gi * GROUP:n_hi + min((gi + 1) * GROUP, n_lo)], 3)
+        scales.append(s)
+        ql.append(q)
+    qh = np.concatenate(qh) if qh else np.zeros(0, np.int8)
+    ql = np.concatenate(ql) if ql else np.zeros(0, np.int8)
+    return qh, ql, np.array(scales, dtype=np.float16)
+
+
+def dequantize_hadamard_latent(qh, ql, scales, r: int) -> np.ndarray:
+    """Codes times their group's fp16 scale (exact in fp32), in channel order."""
+    sp = hadamard_split(r)
+    out = np.zeros(r, np.float64)
+    for i in range(sp["n_hi"]):
+        out[i] = np.float64(scales[i // GROUP]) * int(qh[i])
+    for j in range(sp["n_lo"]):
+        out[sp["n_hi"] + j] = np.float64(scales[sp["g_hi"] + j // GROUP]) * int(ql[j])
+    return out
+
+
+def pack_int3(codes) -> np.ndarray:
+    """3-bit two's-complement codes in [-4, 3], eight per three bytes: code i of a group of
+    eight in bits [3i, 3i+3) of a little-endian 24-bit word; a short tail is padded with 0."""
+    codes = np.asarray(codes, dtype=np.int64)
+    assert codes.size == 0 or (codes.min() >= -4 and codes.max() <= 3)
+    n = codes.size
+    padded = np.zeros(-(-n // 8) * 8, np.int64)
+    padded[:n] = codes
+    out = []
+    for k in range(0, padded.size, 8):
+        word = 0
+        for i in range(8):
+            word |= (int(padded[k + i]) & 7) << (3 * i)
+        out += [word & 0xFF, (word >> 8) & 0xFF, (word >> 16) & 0xFF]
+    return np.array(out, dtype=np.uint8)
+
+
+def unpack_int3(packed, n: int) -> np.ndarray:
+    """Inverse of pack_int3: the first n codes."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    out = []
+    for k in range(0, packed.size, 3):
+        word = int(packed[k]) | (int(packed[k + 1]) << 8) | (int(packed[k + 2]) << 16)
+        for i in range(8):
+            v = (word >> (3 * i)) & 7
+            out.append(v - 8 if v >= 4 else v)
+    return np.array(out[:n], dtype=np.int8)
 
 
 def pack_int4(codes) -> np.ndarray:
