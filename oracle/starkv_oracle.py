@@ -36,6 +36,9 @@ Readings where the pages are silent (each is listed again in the design notes):
     the even channel.  int8 channels: the first ceil(r/4).
   * RoPE: half-split (rotate-half) form, theta_j = base^(-2j/d), 0-based positions, the
     decode query at position L-1.  Output fp32-comparable fp64.
+  * The pages' own assignment [S2] (keys head-wise, values joint) is decode_attention_hybrid;
+    the pages' weight absorption [S2] with per-head values gives each query head its own
+    M_h = B_v,g(h) W_o,h (absorb_output_weights, decode_attention_absorbed).
   * The pages' own quantiser [S3] (block-wise Hadamard, 4-bit outliers, 3-bit inliers):
     outlier block = the leading ceil(r/5) channels; each block is rotated by normalised
     Sylvester Hadamard matrices, one per set bit of its size (largest first), the transform
