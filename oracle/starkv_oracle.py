@@ -53,6 +53,7 @@ import math
 import numpy as np
 
 F32, BF16, MIXED = "f32", "bf16", "mixed"
+HAD43 = "had43"  # the pages' own format: block-wise Hadamard, 4-bit outliers, 3-bit inliers
 GROUP = 32
 
 
@@ -161,6 +162,8 @@ def page_layout(fmt: str, key_rank: int, value_ranks, page_tokens: int = 64) -> 
       f32:   values  (4 B/channel)
       bf16:  values  (2 B/channel)
       mixed: int8 codes (n8 B) | packed int4 codes (nb4 B) | fp16 scales (2*(g8+g4) B)
+      had43: packed 4-bit codes (nb_hi B) | packed 3-bit codes (nb_lo B) | fp16 scales
+             (2*(g_hi+g_lo) B), for latents of factors rotated by rotate_factors [S3]
     Every block starts on a 16-byte boundary."""
     ranks = [int(key_rank)] + [int(r) for r in value_ranks]
     off = 0
@@ -190,6 +193,15 @@ def page_layout(fmt: str, key_rank: int, value_ranks, page_tokens: int = 64) -> 
             s["i4"] = place(page_tokens * sp["nb4"])
             s["sc"] = place(page_tokens * 2 * (sp["g8"] + sp["g4"]))
             token_bytes += sp["n8"] + sp["nb4"] + 2 * (sp["g8"] + sp["g4"])
+        elif fmt == HAD43:
+            sp = hadamard_split(r)
+            s.update(sp)
+            s["nb_hi"] = -(-sp["n_hi"] // 2)
+            s["nb_lo"] = 3 * -(-sp["n_lo"] // 8)
+            s["hi"] = place(page_tokens * s["nb_hi"])
+            s["lo"] = place(page_tokens * s["nb_lo"])
+            s["sc"] = place(page_tokens * 2 * (sp["g_hi"] + sp["g_lo"]))
+            token_bytes += s["nb_hi"] + s["nb_lo"] + 2 * (sp["g_hi"] + sp["g_lo"])
         else:
             raise ValueError(fmt)
         segs.append(s)
@@ -438,6 +450,15 @@ def encode_token(page: np.ndarray, layout: dict, li: int, slot: int, c) -> None:
         o = seg["plain"] + slot * seg["pitch"]
         hi = (bf16_rne(c).view(np.uint32) >> 16).astype(np.uint16)
         page[o:o + 2 * r] = hi.view(np.uint8)
+    elif fmt == HAD43:
+        qh, ql, sc = quantize_hadamard_latent(c, r)
+        o = seg["hi"] + slot * seg["nb_hi"]
+        page[o:o + seg["nb_hi"]] = pack_int4(qh)
+        o = seg["lo"] + slot * seg["nb_lo"]
+        page[o:o + seg["nb_lo"]] = pack_int3(ql)
+        ns = seg["g_hi"] + seg["g_lo"]
+        o = seg["sc"] + slot * 2 * ns
+        page[o:o + 2 * ns] = sc.view(np.uint8)
     else:
         q8, q4, sc = quantize_latent(c, r)
         o = seg["i8"] + slot * seg["n8"]
@@ -461,6 +482,15 @@ def decode_token(page: np.ndarray, layout: dict, li: int, slot: int) -> np.ndarr
         o = seg["plain"] + slot * seg["pitch"]
         hi = page[o:o + 2 * r].copy().view(np.uint16).astype(np.uint32) << 16
         return hi.view(np.float32).astype(np.float64)
+    if fmt == HAD43:
+        o = seg["hi"] + slot * seg["nb_hi"]
+        qh = unpack_int4(page[o:o + seg["nb_hi"]], seg["n_hi"])
+        o = seg["lo"] + slot * seg["nb_lo"]
+        ql = unpack_int3(page[o:o + seg["nb_lo"]], seg["n_lo"])
+        ns = seg["g_hi"] + seg["g_lo"]
+        o = seg["sc"] + slot * 2 * ns
+        sc = page[o:o + 2 * ns].copy().view(np.float16)
+        return dequantize_hadamard_latent(qh, ql, sc, r)
     o = seg["i8"] + slot * seg["n8"]
     q8 = page[o:o + seg["n8"]].copy().view(np.int8)
     o = seg["i4"] + slot * seg["nb4"]

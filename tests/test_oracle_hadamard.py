@@ -121,3 +121,29 @@ def test_average_bits_at_the_pages_split():
     sp = O.hadamard_split(r)
     bits = (4 * sp["n_hi"] + 3 * sp["n_lo"]) / r
     assert bits == O.two_level_bits(0.2, 4, 3) == pytest.approx(3.2)
+
+
+def test_page_layout_of_the_hadamard_format():
+    L = O.page_layout(O.HAD43, 100, [40, 13])
+    k = L["segs"][0]
+    # rank 100: 20 outlier channels (10 bytes of 4-bit codes), 80 inlier channels (30 bytes
+    # of 3-bit codes), 1 + 3 fp16 scales
+    assert (k["nb_hi"], k["nb_lo"], k["g_hi"] + k["g_lo"]) == (10, 30, 4)
+    assert L["token_bytes"] == (10 + 30 + 8) + (4 + 12 + 4) + (2 + 6 + 4)
+    for seg in L["segs"]:
+        for key in ("hi", "lo", "sc"):
+            assert seg[key] % 16 == 0
+
+
+def test_page_roundtrip_of_the_hadamard_format():
+    g = np.random.default_rng(8)
+    ranks = [100, 40, 13]
+    L = O.page_layout(O.HAD43, ranks[0], ranks[1:])
+    page = np.zeros(L["page_bytes"], np.uint8)
+    for slot in (0, 17, 63):
+        for li, r in enumerate(ranks):
+            c = (g.standard_normal(r) * np.exp(-np.arange(r) / 16.0)).astype(np.float32)
+            rot = (c.astype(np.float64) @ O.hadamard_transform(r)).astype(np.float32)
+            O.encode_token(page, L, li, slot, rot)
+            want = O.dequantize_hadamard_latent(*O.quantize_hadamard_latent(rot, r), r)
+            np.testing.assert_array_equal(O.decode_token(page, L, li, slot), want)
