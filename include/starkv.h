@@ -207,7 +207,10 @@ STARKV_API starkv_status starkv_dequant(const starkv_layout* lay, const void* ca
  *   workspace  device, >= decode_workspace_bytes of starkv_alloc for this batch/max_pages
  * Two launches: a persistent split kernel (tcgen05 K reconstruction into TMEM, RoPE,
  * online softmax, latent P.C_v, one partial per 128-token tile and query head) and a
- * combine kernel (log-sum-exp merge of the partials, then o = a B_v). */
+ * combine kernel (log-sum-exp merge of the partials, then o = a B_v).
+ * STARKV_ERR_UNSUPPORTED, with nothing launched, when the split kernel's shared-memory plan
+ * does not fit the device (fp32 latents with 8 query heads per KV head, for one);
+ * starkv_decode_plan_query answers that on the host beforehand. */
 STARKV_API starkv_status starkv_decode_attention(const starkv_layout* lay, const void* q, const void* cache,
                                       int64_t num_pages, const int32_t* block_table,
                                       int32_t max_pages, const int32_t* seq_lens, int32_t batch,
@@ -215,6 +218,30 @@ STARKV_API starkv_status starkv_decode_attention(const starkv_layout* lay, const
                                       size_t rope_table_bytes, float* out, void* workspace,
                                       size_t workspace_bytes, const starkv_decode_opts* opts,
                                       int32_t* dev_status, starkv_stream_t stream);
+
+/* Launch shape that starkv_decode_attention / starkv_decode_partials choose for a layout,
+ * batch and block-table width on a device with ``num_sms`` SMs and ``smem_per_block`` bytes
+ * of opt-in shared memory per block (148 and 232448 on a B200).  Host only, pure: the decode
+ * calls make the same choice with the current device's figures. */
+typedef struct {
+  int32_t cta_group;     /* 1: one CTA per 128-token tile; 2: a CTA pair per 256-token tile  */
+  int32_t key_mode;      /* int8/int4 keys: 1 = dequantised operand resident per tile, 2 =
+                            codes staged per tile and the operand streamed through the ring,
+                            0 = codes read from global memory; 0 for f32/bf16 (TMA ring)      */
+  int32_t chunk_cols;    /* columns of K (KV heads x d) reconstructed per MMA chunk          */
+  int32_t n_chunks;      /* chunks per tile                                                  */
+  int32_t n_ranges;      /* work units a tile's chunks are split into                        */
+  int32_t stages;        /* operand ring stages                                              */
+  int32_t value_buffers; /* value-latent buffers (double-buffered page pairs)                */
+  int32_t smem_bytes;    /* dynamic shared memory per CTA                                    */
+  int32_t grid;          /* CTAs launched (pairs are further capped at those co-resident)    */
+  int32_t work_units;    /* (tile group, sequence, range) units of the persistent loop        */
+} starkv_decode_plan;
+
+STARKV_API starkv_status starkv_decode_plan_query(const starkv_layout* lay, int32_t batch,
+                                                  int32_t max_pages, const starkv_decode_opts* opts,
+                                                  int32_t num_sms, int64_t smem_per_block,
+                                                  starkv_decode_plan* out);
 
 /* The split step of starkv_decode_attention alone: one partial record per (sequence b,
  * query head h, 128-token tile t) in ``workspace``, at float offset

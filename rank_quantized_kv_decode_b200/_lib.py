@@ -48,6 +48,12 @@ class DecodeOpts(ctypes.Structure):
     _fields_ = [("max_ctas", i32), ("n_ranges", i32), ("timeout_ms", i32), ("cta_group", i32)]
 
 
+class DecodePlan(ctypes.Structure):
+    _fields_ = [("cta_group", i32), ("key_mode", i32), ("chunk_cols", i32), ("n_chunks", i32),
+                ("n_ranges", i32), ("stages", i32), ("value_buffers", i32), ("smem_bytes", i32),
+                ("grid", i32), ("work_units", i32)]
+
+
 EXPORTS = {
     "starkv_layout_init": (i32, [ctypes.POINTER(Config), ctypes.POINTER(Layout)]),
     "starkv_alloc": (i32, [ctypes.POINTER(Layout), i64, i32, i32, i32, ctypes.POINTER(Sizes)]),
@@ -63,6 +69,8 @@ EXPORTS = {
                                       vp]),
     "starkv_decode_partials": (i32, [ctypes.POINTER(Layout), vp, vp, i64, vp, i32, vp, i32, vp, vp,
                                      sz, vp, sz, ctypes.POINTER(DecodeOpts), vp, vp]),
+    "starkv_decode_plan_query": (i32, [ctypes.POINTER(Layout), i32, i32, ctypes.POINTER(DecodeOpts),
+                                       i32, i64, ctypes.POINTER(DecodePlan)]),
     "starkv_decode_combine": (i32, [ctypes.POINTER(Layout), vp, i32, i32, vp, vp, sz, vp, vp]),
     "starkv_decode_attention_noalloc": (i32, [ctypes.POINTER(Layout), vp, vp, i64, vp, i32, vp, i32,
                                               vp, vp, vp, sz, vp, ctypes.POINTER(DecodeOpts), vp,

@@ -117,6 +117,17 @@ def decode_attention_noalloc(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rop
         ctypes.byref(opts), _ptr(status), _stream(stream)), "starkv_decode_attention_noalloc")
 
 
+def decode_plan(lay, batch: int, max_pages: int, max_ctas: int = 0, n_ranges: int = 0,
+                cta_group: int = 0, num_sms: int = 148, smem_per_block: int = 232448) -> L.DecodePlan:
+    """The launch shape the decode calls choose (host only; defaults are a B200's figures)."""
+    opts = L.DecodeOpts(max_ctas, n_ranges, 0, cta_group)
+    out = L.DecodePlan()
+    L.check(L.load().starkv_decode_plan_query(ctypes.byref(lay), batch, max_pages,
+                                              ctypes.byref(opts), num_sms, smem_per_block,
+                                              ctypes.byref(out)), "starkv_decode_plan_query")
+    return out
+
+
 def decode_partials(lay, q, cache, block_table, seq_lens, Bk_t, rope_table, workspace, status,
                     max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
                     cta_group: int = 0, stream=None) -> None:

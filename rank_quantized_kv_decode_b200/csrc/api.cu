@@ -419,57 +419,22 @@ starkv_status starkv_append(const starkv_layout* lay, const void* x, int32_t n_t
   return STARKV_OK;
 }
 
-static starkv_status plan_decode(const starkv_layout* lay, const void* q, const void* cache,
-                                 int64_t num_pages, const int32_t* block_table, int32_t max_pages,
-                                 const int32_t* seq_lens, int32_t batch, const void* Bk_t,
-                                 const float* Bv, const void* rope_table, size_t rope_table_bytes,
-                                 float* out, void* workspace, size_t workspace_bytes,
-                                 const starkv_decode_opts* opts, int32_t* dev_status, bool split,
-                                 bool combine, DecodeParams& p, CUtensorMap& tmA, CUtensorMap& tmB,
-                                 int& grid) {
-  starkv_status st = check_layout(lay);
-  if (st != STARKV_OK) return st;
-  if (batch < 0 || max_pages < 1 || (split && num_pages < 1))
-    return fail(STARKV_ERR_INVALID_ARG, "batch < 0, or max_pages/num_pages < 1");
-  if (batch == 0) return STARKV_OK;
-  if (!seq_lens || !workspace) return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
-  if (split && (!q || !cache || !block_table || !Bk_t || !rope_table || !dev_status))
-    return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
-  if (combine && (!Bv || !out)) return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
-  if (split && ((reinterpret_cast<uintptr_t>(cache) | reinterpret_cast<uintptr_t>(Bk_t) |
-                 reinterpret_cast<uintptr_t>(rope_table)) & 15))
-    return fail(STARKV_ERR_INVALID_ARG, "cache, Bk_t and rope_table must be 16-byte aligned");
-  if (reinterpret_cast<uintptr_t>(workspace) & 15)
-    return fail(STARKV_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
-  if (max_pages > (1 << 24)) return fail(STARKV_ERR_INVALID_ARG, "max_pages too large");
-  if (split && rope_table_bytes < rope_bytes(lay, max_pages))
-    return fail(STARKV_ERR_WORKSPACE, "rope table smaller than needed for max_pages");
+// Launch shape of the split kernel for a layout, batch and block-table width on a device with
+// `sms` SMs and `smem_optin` bytes of opt-in shared memory per block: CTA pairing, chunking,
+// work units, the int8/int4 key-operand mode and the shared-memory plan.  Host only, pure:
+// fills the shape fields of `p` (it zeroes `p` first) and the grid.
+static starkv_status plan_shape(const starkv_layout* lay, int32_t batch, int32_t max_pages,
+                                const starkv_decode_opts* opts, int sms, size_t smem_optin,
+                                DecodeParams& p, int& grid) {
   const starkv_config& c = lay->cfg;
-  const int tiles_max = tiles_for(max_pages);
-  const int rec = record_floats(lay);
-  const size_t ws_need = static_cast<size_t>(batch) * c.n_q_heads * tiles_max * rec * sizeof(float);
-  if (workspace_bytes < ws_need) return fail(STARKV_ERR_WORKSPACE, "decode workspace too small");
-  DevInfo info;
-  st = current_device(info);
-  if (st != STARKV_OK) return st;
   std::memset(&p, 0, sizeof(p));
   const int fmt = c.fmt, es = elem_size(fmt), d = c.head_dim;
-  p.cache = reinterpret_cast<const uint8_t*>(cache);
-  p.num_pages = num_pages;
-  p.page_bytes = lay->page_bytes;
-  p.block_table = block_table;
+  const int tiles_max = tiles_for(max_pages);
   p.max_pages = max_pages;
-  p.seq_lens = seq_lens;
   p.batch = batch;
-  p.q = q;
-  p.Bv = Bv;
-  p.rope = reinterpret_cast<const float2*>(rope_table);
   p.rope_tiles = rope_tiles_for(max_pages);
-  p.ws = reinterpret_cast<float*>(workspace);
   p.tiles_max = tiles_max;
-  p.rec = rec;
-  p.out = out;
-  p.status = dev_status;
+  p.rec = record_floats(lay);
   const int timeout_ms = (opts && opts->timeout_ms > 0) ? opts->timeout_ms : 4000;
   p.timeout_ns = static_cast<unsigned long long>(timeout_ms) * 1000000ull;
   p.H = c.n_q_heads;
@@ -482,11 +447,12 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   // fp32 latents keep hi/lo copies of both operands in shared memory: 128-column chunks
   p.NC = ncols >= 256 ? (fmt == STARKV_FMT_F32 ? 128 : 256) : ncols;
   p.n_chunks = ceil_div(ncols, p.NC);
+  if (p.n_chunks > kMaxChunks) return fail(STARKV_ERR_UNSUPPORTED, "more K column chunks than supported");
   p.kb_count = ceil_div(c.key_rank * es, kKBytes);
   // CTA pairs (one cluster per 256-token tile) for 16-bit operands and 256-column chunks
   const int want_cg = opts ? opts->cta_group : 0;
   if (want_cg < 0 || want_cg > 2) return fail(STARKV_ERR_INVALID_ARG, "cta_group must be 0, 1 or 2");
-  const bool pair_ok = fmt != STARKV_FMT_F32 && p.NC == 256 && info.sms >= 2;
+  const bool pair_ok = fmt != STARKV_FMT_F32 && p.NC == 256 && sms >= 2;
   if (want_cg == 2 && !pair_ok)
     return fail(STARKV_ERR_UNSUPPORTED, "CTA pairs need bf16 or int8/int4 latents and 256-column chunks");
   // the streamed int8/int4 operand (key rank > 256, dequantised per ring stage) ran slower on
@@ -495,7 +461,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   const bool pair_default = pair_ok && !(fmt == STARKV_FMT_MIXED && p.kb_count > 4);
   p.cta_group = want_cg == 2 ? 2 : (want_cg == 1 ? 1 : (pair_default ? 2 : 1));
   const int CG = p.cta_group;
-  int grid_cap = info.sms;
+  int grid_cap = sms;
   if (opts && opts->max_ctas > 0 && opts->max_ctas < grid_cap) grid_cap = opts->max_ctas;
   grid_cap = std::max(CG, grid_cap / CG * CG);
   const long long group_tiles = ceil_div(tiles_max, CG);
@@ -562,7 +528,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   // shared-memory plan: ring stages of (A k-block, B k-block), value buffers, small arrays
   p.vslot = (vmax + 127) / 128 * 128;
   const size_t bstage = static_cast<size_t>(p.NC / CG) * kKBytes;
-  const size_t limit = std::min<size_t>(decode_smem_limit(), info.smem_optin);
+  const size_t limit = std::min<size_t>(decode_smem_limit(), smem_optin);
   bool planned = false;
   const int plans[][2] = {{6, 2}, {6, 1}, {5, 2}, {5, 1}, {4, 2}, {4, 1}, {3, 2}, {3, 1}, {2, 1}};
   for (int mi = 0; mi < n_modes && !planned; ++mi)
@@ -622,6 +588,58 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   }
   if (!planned) return fail(STARKV_ERR_UNSUPPORTED, "value latents of one chunk do not fit in shared memory");
 
+  grid = static_cast<int>(std::min<long long>(units * CG, grid_cap));
+  return STARKV_OK;
+}
+
+static starkv_status plan_decode(const starkv_layout* lay, const void* q, const void* cache,
+                                 int64_t num_pages, const int32_t* block_table, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t batch, const void* Bk_t,
+                                 const float* Bv, const void* rope_table, size_t rope_table_bytes,
+                                 float* out, void* workspace, size_t workspace_bytes,
+                                 const starkv_decode_opts* opts, int32_t* dev_status, bool split,
+                                 bool combine, DecodeParams& p, CUtensorMap& tmA, CUtensorMap& tmB,
+                                 int& grid) {
+  starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  if (batch < 0 || max_pages < 1 || (split && num_pages < 1))
+    return fail(STARKV_ERR_INVALID_ARG, "batch < 0, or max_pages/num_pages < 1");
+  if (batch == 0) return STARKV_OK;
+  if (!seq_lens || !workspace) return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
+  if (split && (!q || !cache || !block_table || !Bk_t || !rope_table || !dev_status))
+    return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
+  if (combine && (!Bv || !out)) return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
+  if (split && ((reinterpret_cast<uintptr_t>(cache) | reinterpret_cast<uintptr_t>(Bk_t) |
+                 reinterpret_cast<uintptr_t>(rope_table)) & 15))
+    return fail(STARKV_ERR_INVALID_ARG, "cache, Bk_t and rope_table must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(workspace) & 15)
+    return fail(STARKV_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (max_pages > (1 << 24)) return fail(STARKV_ERR_INVALID_ARG, "max_pages too large");
+  if (split && rope_table_bytes < rope_bytes(lay, max_pages))
+    return fail(STARKV_ERR_WORKSPACE, "rope table smaller than needed for max_pages");
+  const starkv_config& c = lay->cfg;
+  const int tiles_max = tiles_for(max_pages);
+  const int rec = record_floats(lay);
+  const size_t ws_need = static_cast<size_t>(batch) * c.n_q_heads * tiles_max * rec * sizeof(float);
+  if (workspace_bytes < ws_need) return fail(STARKV_ERR_WORKSPACE, "decode workspace too small");
+  DevInfo info;
+  st = current_device(info);
+  if (st != STARKV_OK) return st;
+  st = plan_shape(lay, batch, max_pages, opts, info.sms, info.smem_optin, p, grid);
+  if (st != STARKV_OK) return st;
+  const int fmt = c.fmt, es = elem_size(fmt), CG = p.cta_group;
+  const int ncols = c.n_kv_heads * c.head_dim;
+  p.cache = reinterpret_cast<const uint8_t*>(cache);
+  p.num_pages = num_pages;
+  p.page_bytes = lay->page_bytes;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.q = q;
+  p.Bv = Bv;
+  p.rope = reinterpret_cast<const float2*>(rope_table);
+  p.ws = reinterpret_cast<float*>(workspace);
+  p.out = out;
+  p.status = dev_status;
   std::memset(&tmA, 0, sizeof(tmA));
   std::memset(&tmB, 0, sizeof(tmB));
   if (!split) return STARKV_OK;
@@ -648,7 +666,32 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
     st = encode(&tmB, dt, 2, Bk_t, dims, strides, box);
     if (st != STARKV_OK) return st;
   }
-  grid = static_cast<int>(std::min<long long>(units * CG, grid_cap));
+  return STARKV_OK;
+}
+
+starkv_status starkv_decode_plan_query(const starkv_layout* lay, int32_t batch, int32_t max_pages,
+                                       const starkv_decode_opts* opts, int32_t num_sms,
+                                       int64_t smem_per_block, starkv_decode_plan* out) {
+  starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  if (!out) return fail(STARKV_ERR_INVALID_ARG, "out is NULL");
+  if (batch < 1 || max_pages < 1 || max_pages > (1 << 24) || num_sms < 1 || smem_per_block < 0)
+    return fail(STARKV_ERR_INVALID_ARG, "batch, max_pages and num_sms must be >= 1");
+  DecodeParams p;
+  int grid = 0;
+  st = plan_shape(lay, batch, max_pages, opts, num_sms, static_cast<size_t>(smem_per_block), p, grid);
+  if (st != STARKV_OK) return st;
+  std::memset(out, 0, sizeof(*out));
+  out->cta_group = p.cta_group;
+  out->key_mode = p.a_resident;
+  out->chunk_cols = p.NC;
+  out->n_chunks = p.n_chunks;
+  out->n_ranges = p.n_ranges;
+  out->stages = p.stages;
+  out->value_buffers = p.nvb;
+  out->smem_bytes = static_cast<int32_t>(p.smem_bytes);
+  out->grid = grid;
+  out->work_units = p.total_units;
   return STARKV_OK;
 }
 
