@@ -303,6 +303,11 @@ static starkv_status store_common(const starkv_layout* lay, int32_t n_tok, const
     return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
   std::memset(&sp, 0, sizeof(sp));
   fill_store(sp, lay);
+  // the store and read-back kernels number their warps (token x chunk, token x latent) in
+  // 32-bit integers
+  const int64_t warps = static_cast<int64_t>(n_tok) * std::max(sp.chunks_per_token, lay->n_latents);
+  if (warps > (int64_t(1) << 31) - 256)
+    return fail(STARKV_ERR_INVALID_ARG, "n_tok too large for one call; split the tokens");
   sp.cache = reinterpret_cast<uint8_t*>(cache);
   sp.num_pages = num_pages;
   sp.page_bytes = lay->page_bytes;

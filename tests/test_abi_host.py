@@ -135,3 +135,16 @@ def test_tampered_layout_rejected(lib):
     lay.page_bytes += 16
     s = L.Sizes()
     assert lib.starkv_alloc(ctypes.byref(lay), 4, 1, 4, 0, ctypes.byref(s)) == L.ERR_INVALID_ARG
+
+
+def test_store_rejects_token_counts_past_32_bit_warp_numbering(lib):
+    # key rank 2048 int8/int4: 64 chunks per token for the key alone, so ~33.5 M tokens would
+    # number warps past 2^31; refused before any device call (the pointers are never used)
+    lay = api.layout_init(api.make_config(8, 1, 128, 4096, 2048, [128], "mixed", 10000.0))
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.starkv_quant_pack(ctypes.byref(lay), fake, 40_000_000, fake, fake, fake, 1, 1, fake,
+                               1, fake, None)
+    assert st == L.ERR_INVALID_ARG and b"split the tokens" in lib.starkv_last_error()
+    st = lib.starkv_dequant(ctypes.byref(lay), fake, 1, fake, fake, 40_000_000, fake, 1, 1, fake,
+                            fake, None)
+    assert st == L.ERR_INVALID_ARG
