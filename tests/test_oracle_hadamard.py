@@ -8,11 +8,14 @@ Methodology §3: block-wise Hadamard rotation of an outlier and an inlier block,
 * a single spike in a block of 2^k channels is spread to 2^-k/2 of its height (the
   smoothing the rotation is there for);
 * the 3-bit packing: a hand-worked word, every code at every position, random lengths;
+* hand-worked 3-bit groups (tests/golden/quant_groups_3bit.txt): ties to even, a scale that
+  rounds down to an fp16 subnormal, saturation, the zero group;
 * quantisation error at most half a scale step per channel, groups restarting at the block
   boundary, and the format's average of 3.2 bits per channel (scales excluded) at the
   pages' 20 % / 80 % split.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -147,3 +150,35 @@ def test_page_roundtrip_of_the_hadamard_format():
             O.encode_token(page, L, li, slot, rot)
             want = O.dequantize_hadamard_latent(*O.quantize_hadamard_latent(rot, r), r)
             np.testing.assert_array_equal(O.decode_token(page, L, li, slot), want)
+
+
+def _golden_3bit():
+    rows = []
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "quant_groups_3bit.txt")
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            bits, vals, s16, codes = [p.strip() for p in line.split(";")]
+            vals = [float.fromhex(v) if "0x" in v else float(v) for v in vals.split()]
+            rows.append((int(bits), np.array(vals, np.float32), int(s16, 16), [int(c) for c in codes.split()]))
+    return rows
+
+
+@pytest.mark.parametrize("row", _golden_3bit())
+def test_quantize_3bit_group_golden(row):
+    bits, vals, s16_bits, codes = row
+    assert bits == 3
+    s16, q = O.quantize_group(vals, bits)
+    assert int(np.array(s16, np.float16).view(np.uint16)) == s16_bits
+    assert q.tolist() == codes
+    # the same group placed at the start of a rank-40 latent's inlier block, behind an
+    # all-zero outlier block (scale 0), comes out of the format's quantiser unchanged
+    sp = O.hadamard_split(40)
+    c = np.zeros(40, np.float32)
+    c[sp["n_hi"]:sp["n_hi"] + len(vals)] = vals
+    qh, ql, sc = O.quantize_hadamard_latent(c, 40)
+    assert not qh.any() and not sc[:sp["g_hi"]].view(np.uint16).any()
+    assert ql[:len(vals)].tolist() == codes
+    assert int(sc[sp["g_hi"]:sp["g_hi"] + 1].view(np.uint16)[0]) == s16_bits
