@@ -74,7 +74,12 @@ typedef enum {
 typedef enum {
   STARKV_FMT_F32 = 0,  /* latents stored as fp32; tf32 tensor cores for K = C_k B_k  */
   STARKV_FMT_BF16 = 1, /* latents stored as bf16 (RNE); bf16 tensor cores             */
-  STARKV_FMT_MIXED = 2 /* int8/int4 codes + fp16 group scales; fp16 tensor cores       */
+  STARKV_FMT_MIXED = 2, /* int8/int4 codes + fp16 group scales; fp16 tensor cores      */
+  STARKV_FMT_HAD43 = 3  /* STAR-KV technical summary, Methodology §3: latents of factors
+                           rotated by a block-wise Hadamard transform, the leading
+                           ceil(r/5) channels as 4-bit codes, the rest as 3-bit codes, fp16
+                           group scales.  Page layout only so far (starkv_layout_init,
+                           starkv_alloc); the device calls return STARKV_ERR_UNSUPPORTED */
 } starkv_fmt;
 
 /* Model/cache description (host struct, POD). */
@@ -92,7 +97,16 @@ typedef struct {
 
 /* One latent's place in a page.  Latent 0 is the key latent, latent 1+g the value latent
  * of KV head g.  Each block is token-major ([token][...]) and starts on a 16-byte
- * boundary; absent blocks have offset -1. */
+ * boundary; absent blocks have offset -1.  The quantised formats have two channel blocks,
+ * the leading (more precise) one and the rest; in had43 the fields named for int8/int4 hold
+ * them as follows:
+ *   n8, g8   4-bit channels [0, n8), n8 = ceil(r/5), and their scale groups ceil(n8/32)
+ *   n4, g4   3-bit channels [n8, r) and their scale groups ceil(n4/32)
+ *   pitch    bytes per token of the packed 4-bit codes, ceil(n8/2), at off_i8; channel 2i
+ *            in the low nibble of byte i, 2i+1 in the high nibble
+ *   nb4      bytes per token of the packed 3-bit codes, 3*ceil(n4/8), at off_i4; each 3
+ *            bytes hold 8 codes c_0..c_7 as the little-endian 24-bit word sum_i (c_i & 7) 8^i
+ *   off_sc   fp16 scales [page_tokens][g8+g4], 4-bit groups first */
 typedef struct {
   int32_t rank;  /* channels r                                                          */
   int32_t col;   /* first column of this latent in the concatenated projection

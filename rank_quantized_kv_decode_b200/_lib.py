@@ -12,7 +12,7 @@ MAX_KV_HEADS = 64
 GROUP = 32
 TILE_TOKENS = 128
 
-FMT = {"f32": 0, "bf16": 1, "mixed": 2}
+FMT = {"f32": 0, "bf16": 1, "mixed": 2, "had43": 3}
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BOUNDS, DEV_TIMEOUT = 1, 2

@@ -124,6 +124,13 @@ starkv_status check_layout(const starkv_layout* lay) {
   return STARKV_OK;
 }
 
+// The formats the kernels implement (the had43 page layout has no kernels yet).
+starkv_status check_device_format(const starkv_layout* lay) {
+  if (lay->cfg.fmt == STARKV_FMT_HAD43)
+    return fail(STARKV_ERR_UNSUPPORTED, "the had43 format has a page layout but no kernels yet");
+  return STARKV_OK;
+}
+
 // Split-K plan of the projection: about one CTA per SM of a B200 (148), every split non-empty.
 constexpr int kProjCtaTarget = 148;
 void proj_plan(const starkv_layout* lay, int n_tok, int& kb_total, int& kb_per_split, int& nsplit) {
@@ -193,7 +200,8 @@ starkv_status starkv_layout_init(const starkv_config* cfg, starkv_layout* out) {
     return fail(STARKV_ERR_INVALID_ARG, "d_model must be a positive multiple of 16");
   if (c.key_rank < 16 || c.key_rank % 16 != 0 || c.key_rank > 2048)
     return fail(STARKV_ERR_INVALID_ARG, "key_rank must be a multiple of 16 in [16, 2048]");
-  if (c.fmt != STARKV_FMT_F32 && c.fmt != STARKV_FMT_BF16 && c.fmt != STARKV_FMT_MIXED)
+  if (c.fmt != STARKV_FMT_F32 && c.fmt != STARKV_FMT_BF16 && c.fmt != STARKV_FMT_MIXED &&
+      c.fmt != STARKV_FMT_HAD43)
     return fail(STARKV_ERR_INVALID_ARG, "unknown latent format");
   if (c.page_tokens != kPage) return fail(STARKV_ERR_UNSUPPORTED, "page_tokens must be 64");
   if (!(c.rope_theta > 1.0) || !std::isfinite(c.rope_theta))
@@ -235,6 +243,17 @@ starkv_status starkv_layout_init(const starkv_config* cfg, starkv_layout* out) {
       s.off_i4 = place(static_cast<int64_t>(kPage) * s.nb4);
       s.off_sc = place(static_cast<int64_t>(kPage) * 2 * (s.g8 + s.g4));
       token_bytes += s.n8 + s.nb4 + 2 * (s.g8 + s.g4);
+    } else if (c.fmt == STARKV_FMT_HAD43) {
+      s.n8 = (r + 4) / 5;  // the outlier block: a fifth of the channels, rounded up
+      s.n4 = r - s.n8;
+      s.g8 = (s.n8 + STARKV_GROUP - 1) / STARKV_GROUP;
+      s.g4 = (s.n4 + STARKV_GROUP - 1) / STARKV_GROUP;
+      s.pitch = (s.n8 + 1) / 2;
+      s.nb4 = 3 * ((s.n4 + 7) / 8);
+      s.off_i8 = place(static_cast<int64_t>(kPage) * s.pitch);
+      s.off_i4 = place(static_cast<int64_t>(kPage) * s.nb4);
+      s.off_sc = place(static_cast<int64_t>(kPage) * 2 * (s.g8 + s.g4));
+      token_bytes += s.pitch + s.nb4 + 2 * (s.g8 + s.g4);
     } else {
       const int es = elem_size(c.fmt);
       s.pitch = r * es;
@@ -296,6 +315,8 @@ static starkv_status store_common(const starkv_layout* lay, int32_t n_tok, const
                                   int32_t max_pages, int32_t batch, void* cache, int64_t num_pages,
                                   int32_t* dev_status, StoreParams& sp) {
   starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  st = check_device_format(lay);
   if (st != STARKV_OK) return st;
   if (n_tok < 0 || max_pages < 1 || batch < 1 || num_pages < 1)
     return fail(STARKV_ERR_INVALID_ARG, "n_tok < 0, or batch/max_pages/num_pages < 1");
@@ -607,6 +628,8 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
                                  int& grid) {
   starkv_status st = check_layout(lay);
   if (st != STARKV_OK) return st;
+  st = check_device_format(lay);
+  if (st != STARKV_OK) return st;
   if (batch < 0 || max_pages < 1 || (split && num_pages < 1))
     return fail(STARKV_ERR_INVALID_ARG, "batch < 0, or max_pages/num_pages < 1");
   if (batch == 0) return STARKV_OK;
@@ -678,6 +701,8 @@ starkv_status starkv_decode_plan_query(const starkv_layout* lay, int32_t batch, 
                                        const starkv_decode_opts* opts, int32_t num_sms,
                                        int64_t smem_per_block, starkv_decode_plan* out) {
   starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  st = check_device_format(lay);
   if (st != STARKV_OK) return st;
   if (!out) return fail(STARKV_ERR_INVALID_ARG, "out is NULL");
   if (batch < 1 || max_pages < 1 || max_pages > (1 << 24) || num_sms < 1 || smem_per_block < 0)

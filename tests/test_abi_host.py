@@ -51,6 +51,8 @@ CASES = [
     ("bf16", 32, 32, 128, 4096, 1024, [16 + (g * 7) % 49 for g in range(32)]),
     ("mixed", 32, 32, 128, 4096, 1024, [16 + (g * 5) % 49 for g in range(32)]),
     ("mixed", 32, 8, 128, 4096, 256, [8, 48, 37, 17, 32, 29, 40, 45]),
+    ("had43", 32, 8, 128, 4096, 256, [8, 48, 37, 17, 32, 29, 40, 45]),
+    ("had43", 4, 4, 64, 256, 64, [1, 2, 13, 64]),
 ]
 
 
@@ -70,6 +72,12 @@ def test_layout_matches_oracle(lib, fmt, H, Hkv, d, dm, rk, rv):
         if fmt == "mixed":
             assert (seg.n8, seg.n4, seg.g8, seg.g4, seg.nb4) == (s["n8"], s["n4"], s["g8"], s["g4"], s["nb4"])
             assert (seg.off_i8, seg.off_i4, seg.off_sc) == (s["i8"], s["i4"], s["sc"])
+            assert seg.off_plain == -1
+        elif fmt == "had43":
+            # the 4-bit outlier block and the 3-bit inlier block in the int8/int4 fields
+            assert (seg.n8, seg.n4, seg.g8, seg.g4) == (s["n_hi"], s["n_lo"], s["g_hi"], s["g_lo"])
+            assert (seg.pitch, seg.nb4) == (s["nb_hi"], s["nb_lo"])
+            assert (seg.off_i8, seg.off_i4, seg.off_sc) == (s["hi"], s["lo"], s["sc"])
             assert seg.off_plain == -1
         else:
             assert seg.off_plain == s["plain"] and seg.pitch == s["pitch"]
@@ -148,3 +156,32 @@ def test_store_rejects_token_counts_past_32_bit_warp_numbering(lib):
     st = lib.starkv_dequant(ctypes.byref(lay), fake, 1, fake, fake, 40_000_000, fake, 1, 1, fake,
                             fake, None)
     assert st == L.ERR_INVALID_ARG
+
+
+def test_had43_layout_is_refused_by_the_device_calls(lib):
+    # the pages' own format has a page layout (above) but no kernels yet: every call that
+    # would launch one refuses it before touching the device (the pointers are never used)
+    lay = api.layout_init(api.make_config(32, 8, 128, 4096, 256, [32] * 8, "had43", 500000.0))
+    s = L.Sizes()
+    assert lib.starkv_alloc(ctypes.byref(lay), 4, 1, 4, 8, ctypes.byref(s)) == L.OK
+    assert s.cache_bytes == 4 * lay.page_bytes
+    fake = ctypes.c_void_p(1 << 20)
+    calls = {
+        "quant_pack": lambda: lib.starkv_quant_pack(ctypes.byref(lay), fake, 1, fake, fake, fake, 1,
+                                                    1, fake, 1, fake, None),
+        "dequant": lambda: lib.starkv_dequant(ctypes.byref(lay), fake, 1, fake, fake, 1, fake, 1, 1,
+                                              fake, fake, None),
+        "append": lambda: lib.starkv_append(ctypes.byref(lay), fake, 1, fake, fake, fake, fake, 1, 1,
+                                            fake, 1, None, fake, 1 << 30, fake, None),
+        "decode_attention": lambda: lib.starkv_decode_attention(
+            ctypes.byref(lay), fake, fake, 1, fake, 1, fake, 1, fake, fake, fake, 1 << 30, fake,
+            fake, 1 << 30, None, fake, None),
+        "decode_combine": lambda: lib.starkv_decode_combine(ctypes.byref(lay), fake, 1, 1, fake,
+                                                            fake, 1 << 30, fake, None),
+        "decode_plan_query": lambda: lib.starkv_decode_plan_query(ctypes.byref(lay), 1, 1, None,
+                                                                  148, 232448,
+                                                                  ctypes.byref(L.DecodePlan())),
+    }
+    for name, call in calls.items():
+        assert call() == L.ERR_UNSUPPORTED, name
+        assert b"had43" in lib.starkv_last_error(), name
