@@ -78,8 +78,9 @@ typedef enum {
   STARKV_FMT_HAD43 = 3  /* STAR-KV technical summary, Methodology §3: latents of factors
                            rotated by a block-wise Hadamard transform, the leading
                            ceil(r/5) channels as 4-bit codes, the rest as 3-bit codes, fp16
-                           group scales.  Page layout only so far (starkv_layout_init,
-                           starkv_alloc); the device calls return STARKV_ERR_UNSUPPORTED */
+                           group scales.  Layout, store (starkv_quant_pack, starkv_append:
+                           bf16 operands) and read-back so far; the decode calls return
+                           STARKV_ERR_UNSUPPORTED */
 } starkv_fmt;
 
 /* Model/cache description (host struct, POD). */
@@ -177,8 +178,8 @@ STARKV_API starkv_status starkv_rope_init(const starkv_layout* lay, int32_t max_
  *   block_table device int32 [batch][max_pages]; token (b, p) goes to page
  *               block_table[b][p / 64], slot p % 64
  *   cache       device, num_pages * page_bytes bytes
- * f32 stores the values, bf16 rounds to nearest even, mixed quantises per group (see
- * starkv_segment) -- bit-exact with the reference definition.  Tokens with a bad page or
+ * f32 stores the values, bf16 rounds to nearest even, mixed and had43 quantise per group
+ * (see starkv_segment) -- bit-exact with the reference definition.  Tokens with a bad page or
  * position are skipped and flagged STARKV_DEV_BOUNDS.  Tokens written by one call must be
  * distinct. */
 STARKV_API starkv_status starkv_quant_pack(const starkv_layout* lay, const float* latents, int32_t n_tok,

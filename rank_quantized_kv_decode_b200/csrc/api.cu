@@ -124,10 +124,10 @@ starkv_status check_layout(const starkv_layout* lay) {
   return STARKV_OK;
 }
 
-// The formats the kernels implement (the had43 page layout has no kernels yet).
-starkv_status check_device_format(const starkv_layout* lay) {
+// The formats the decode kernels implement (had43 has its store and read-back only).
+starkv_status check_decode_format(const starkv_layout* lay) {
   if (lay->cfg.fmt == STARKV_FMT_HAD43)
-    return fail(STARKV_ERR_UNSUPPORTED, "the had43 format has a page layout but no kernels yet");
+    return fail(STARKV_ERR_UNSUPPORTED, "decode of the had43 format is not implemented yet");
   return STARKV_OK;
 }
 
@@ -166,7 +166,8 @@ void fill_store(StoreParams& sp, const starkv_layout* lay) {
     sp.lat[i] = lat_desc(lay->seg[i]);
     sp.chunk_start[i] = static_cast<short>(chunks);
     const starkv_segment& g = lay->seg[i];
-    chunks += lay->cfg.fmt == STARKV_FMT_MIXED ? g.g8 + g.g4 : (g.rank + 31) / 32;
+    const bool grouped = lay->cfg.fmt == STARKV_FMT_MIXED || lay->cfg.fmt == STARKV_FMT_HAD43;
+    chunks += grouped ? g.g8 + g.g4 : (g.rank + 31) / 32;
   }
   sp.chunk_start[lay->n_latents] = static_cast<short>(chunks);
   sp.chunks_per_token = chunks;
@@ -315,8 +316,6 @@ static starkv_status store_common(const starkv_layout* lay, int32_t n_tok, const
                                   int32_t max_pages, int32_t batch, void* cache, int64_t num_pages,
                                   int32_t* dev_status, StoreParams& sp) {
   starkv_status st = check_layout(lay);
-  if (st != STARKV_OK) return st;
-  st = check_device_format(lay);
   if (st != STARKV_OK) return st;
   if (n_tok < 0 || max_pages < 1 || batch < 1 || num_pages < 1)
     return fail(STARKV_ERR_INVALID_ARG, "n_tok < 0, or batch/max_pages/num_pages < 1");
@@ -628,7 +627,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
                                  int& grid) {
   starkv_status st = check_layout(lay);
   if (st != STARKV_OK) return st;
-  st = check_device_format(lay);
+  st = check_decode_format(lay);
   if (st != STARKV_OK) return st;
   if (batch < 0 || max_pages < 1 || (split && num_pages < 1))
     return fail(STARKV_ERR_INVALID_ARG, "batch < 0, or max_pages/num_pages < 1");
@@ -702,7 +701,7 @@ starkv_status starkv_decode_plan_query(const starkv_layout* lay, int32_t batch, 
                                        int64_t smem_per_block, starkv_decode_plan* out) {
   starkv_status st = check_layout(lay);
   if (st != STARKV_OK) return st;
-  st = check_device_format(lay);
+  st = check_decode_format(lay);
   if (st != STARKV_OK) return st;
   if (!out) return fail(STARKV_ERR_INVALID_ARG, "out is NULL");
   if (batch < 1 || max_pages < 1 || max_pages > (1 << 24) || num_sms < 1 || smem_per_block < 0)

@@ -7,6 +7,12 @@
 // The leading ceil(r/4) channels (singular-value order: the outlier channels of STAR-KV
 // technical summary, Methodology §3 "Low-Rank-Aware Mixed-Precision Quantization") are int8,
 // the rest int4, two per byte with the even channel in the low nibble.
+//
+// The pages' own format (had43; same page, Methodology §3 "Low-Rank-Aware Mixed-Precision
+// Quantization"): latents of factors already rotated by the block-wise Hadamard transform;
+// the leading ceil(r/5) channels are 4-bit codes (qmax 7, two per byte as above), the rest
+// 3-bit codes (qmax 3), eight per 3 bytes as the little-endian 24-bit word
+// sum_i (code_i & 7) 8^i; same scale rule, groups of 32 restarting at the 3-bit block.
 #include "internal.cuh"
 
 namespace starkv {
@@ -106,6 +112,38 @@ __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ Stor
     return;
   }
   __half* sc = ts.page ? reinterpret_cast<__half*>(ts.page + d.off2) + ts.slot * d.ng : nullptr;
+  if (p.fmt == STARKV_FMT_HAD43) {
+    const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
+    if (is8) {
+      // 4-bit group cl: channels [32 cl, min(32 cl + 32, n8)), d.pitch packed bytes per token
+      const __half h = group_scale(amax, 7.f);
+      const int nib = quant_code(c, __half2float(h), 7) & 15;
+      const int hi = __shfl_down_sync(0xffffffffu, nib, 1);
+      if (ts.page && in && (i & 1) == 0) {
+        const int byte = nib | ((i + 1 < d.n8 ? hi : 0) << 4);
+        (ts.page + d.off0)[ts.slot * d.pitch + (i >> 1)] = static_cast<uint8_t>(byte);
+      }
+      if (ts.page && lane == 0) sc[cl] = h;
+    } else {
+      // 3-bit group gi: channels n8 + [32 gi, min(32 gi + 32, n4)); lanes 8k..8k+7 form word
+      // k of the group (lanes past n4 hold c = 0, code 0: the padding of the last word)
+      const int gi = cl - d.g8;
+      const __half h = group_scale(amax, 3.f);
+      const int code = quant_code(c, __half2float(h), 3) & 7;
+      uint32_t w = static_cast<uint32_t>(code) << (3 * (lane & 7));
+      w |= __shfl_xor_sync(0xffffffffu, w, 1);
+      w |= __shfl_xor_sync(0xffffffffu, w, 2);
+      w |= __shfl_xor_sync(0xffffffffu, w, 4);
+      if (ts.page && in && (lane & 7) == 0) {
+        uint8_t* dst = ts.page + d.off1 + ts.slot * d.nb4 + 3 * (j >> 3);
+        dst[0] = static_cast<uint8_t>(w);
+        dst[1] = static_cast<uint8_t>(w >> 8);
+        dst[2] = static_cast<uint8_t>(w >> 16);
+      }
+      if (ts.page && lane == 0) sc[d.g8 + gi] = h;
+    }
+    return;
+  }
   if (is8) {
     // int8 group cl: channels [32 cl, min(32 cl + 32, n8))
     const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
@@ -146,6 +184,19 @@ __global__ void __launch_bounds__(128) dequant_kernel(const __grid_constant__ St
         v = reinterpret_cast<const float*>(pg + d.off0 + ts.slot * d.pitch)[i];
       } else if (p.fmt == STARKV_FMT_BF16) {
         v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(pg + d.off0 + ts.slot * d.pitch)[i]);
+      } else if (p.fmt == STARKV_FMT_HAD43) {
+        const __half* sc = reinterpret_cast<const __half*>(pg + d.off2) + ts.slot * d.ng;
+        if (i < d.n8) {
+          const uint8_t byte = (pg + d.off0)[ts.slot * d.pitch + (i >> 1)];
+          const int nib = (i & 1) ? (byte >> 4) : (byte & 15);
+          v = __half2float(sc[i >> 5]) * static_cast<float>((nib ^ 8) - 8);
+        } else {
+          const int j = i - d.n8;
+          const uint8_t* w = pg + d.off1 + ts.slot * d.nb4 + 3 * (j >> 3);
+          const uint32_t word = w[0] | (static_cast<uint32_t>(w[1]) << 8) | (static_cast<uint32_t>(w[2]) << 16);
+          const int code = (word >> (3 * (j & 7))) & 7;
+          v = __half2float(sc[d.g8 + (j >> 5)]) * static_cast<float>((code ^ 4) - 4);
+        }
       } else {
         const __half* sc = reinterpret_cast<const __half*>(pg + d.off2) + ts.slot * d.ng;
         if (i < d.n8) {

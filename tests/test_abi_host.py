@@ -158,26 +158,27 @@ def test_store_rejects_token_counts_past_32_bit_warp_numbering(lib):
     assert st == L.ERR_INVALID_ARG
 
 
-def test_had43_layout_is_refused_by_the_device_calls(lib):
-    # the pages' own format has a page layout (above) but no kernels yet: every call that
-    # would launch one refuses it before touching the device (the pointers are never used)
+def test_had43_decode_is_refused_before_touching_the_device(lib):
+    # the pages' own format has its page layout (above), store and read-back, but no decode
+    # kernel yet: the decode calls refuse it before any device call (the pointers are never
+    # used)
     lay = api.layout_init(api.make_config(32, 8, 128, 4096, 256, [32] * 8, "had43", 500000.0))
     s = L.Sizes()
     assert lib.starkv_alloc(ctypes.byref(lay), 4, 1, 4, 8, ctypes.byref(s)) == L.OK
     assert s.cache_bytes == 4 * lay.page_bytes
     fake = ctypes.c_void_p(1 << 20)
     calls = {
-        "quant_pack": lambda: lib.starkv_quant_pack(ctypes.byref(lay), fake, 1, fake, fake, fake, 1,
-                                                    1, fake, 1, fake, None),
-        "dequant": lambda: lib.starkv_dequant(ctypes.byref(lay), fake, 1, fake, fake, 1, fake, 1, 1,
-                                              fake, fake, None),
-        "append": lambda: lib.starkv_append(ctypes.byref(lay), fake, 1, fake, fake, fake, fake, 1, 1,
-                                            fake, 1, None, fake, 1 << 30, fake, None),
         "decode_attention": lambda: lib.starkv_decode_attention(
             ctypes.byref(lay), fake, fake, 1, fake, 1, fake, 1, fake, fake, fake, 1 << 30, fake,
             fake, 1 << 30, None, fake, None),
+        "decode_partials": lambda: lib.starkv_decode_partials(
+            ctypes.byref(lay), fake, fake, 1, fake, 1, fake, 1, fake, fake, 1 << 30, fake,
+            1 << 30, None, fake, None),
         "decode_combine": lambda: lib.starkv_decode_combine(ctypes.byref(lay), fake, 1, 1, fake,
                                                             fake, 1 << 30, fake, None),
+        "decode_attention_noalloc": lambda: lib.starkv_decode_attention_noalloc(
+            ctypes.byref(lay), fake, fake, 1, fake, 1, fake, 1, fake, fake, fake, 1 << 30, fake,
+            None, fake, None),
         "decode_plan_query": lambda: lib.starkv_decode_plan_query(ctypes.byref(lay), 1, 1, None,
                                                                   148, 232448,
                                                                   ctypes.byref(L.DecodePlan())),
