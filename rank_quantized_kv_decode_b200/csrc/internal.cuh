@@ -11,7 +11,7 @@ constexpr int kTile = STARKV_TILE_TOKENS;  // tokens per decode tile
 constexpr int kPage = 64;                  // tokens per page
 constexpr int kKBytes = 128;               // bytes of K per operand row per k-block
 constexpr int kAStage = kTile * kKBytes;   // 16 KB: one k-block of a 128-row tile
-constexpr int kMaxChunks = 64;             // ceil(64 heads * 128 / 128): fp32 latents use 128-column chunks
+constexpr int kMaxChunks = 32;             // ceil(64 heads * 128 / 256)
 
 // One latent's description for device code (offsets inside a page; page_bytes < 2^31).
 struct LatDesc {
