@@ -65,3 +65,39 @@ def test_two_gloo_ranks():
         assert mx == 0.75
         assert rate == pytest.approx(8 * 4096 * 2 / 0.75)
         assert got == [1] * 16
+
+
+def _leaving_worker(rank, world, port, q):
+    """Rank 1 leaves between steps (it raises before the timing reduction, with nothing in
+    flight); rank 0 must learn of it from its next collective, as an error, not a hang."""
+    import time
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=5))
+    D.max_over_ranks(1.0)  # one step that both ranks complete
+    if rank == 1:
+        q.put((rank, "left", 0.0))
+        raise SystemExit(3)
+    t0 = time.monotonic()
+    try:
+        D.max_over_ranks(2.0)
+        q.put((rank, "no error", time.monotonic() - t0))
+    except Exception as e:  # noqa: BLE001 -- the backend's error type is not part of its API
+        q.put((rank, "error: " + type(e).__name__, time.monotonic() - t0))
+
+
+def test_a_rank_that_leaves_ends_the_others_next_collective_with_an_error():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_leaving_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict((r, (what, dt)) for r, what, dt in [q.get(timeout=120) for _ in range(world)])
+    for p in procs:
+        p.join(timeout=60)
+    assert procs[1].exitcode == 3
+    what, dt = res[0]
+    assert what.startswith("error"), what
+    assert dt < 30.0  # bounded by the process group's 5 s timeout, not a hang
