@@ -717,8 +717,38 @@ def dequantize_rows(q8, q4, scales, r: int) -> np.ndarray:
     return np.concatenate([s8 * q8, s4 * q4], axis=1)
 
 
+def quantize_hadamard_rows(C, r: int):
+    """quantize_hadamard_latent for every row of C (n, r) fp32 (rotated latents):
+    (4-bit codes (n, n_hi), 3-bit codes (n, n_lo), scales (n, g_hi + g_lo))."""
+    C = np.asarray(C, dtype=np.float32)
+    sp = hadamard_split(r)
+    n_hi, n_lo = sp["n_hi"], sp["n_lo"]
+    scales, qh, ql = [], [], []
+    for gi in range(sp["g_hi"]):
+        s, q = _quantize_block(C[:, gi * GROUP:min((gi + 1) * GROUP, n_hi)], 4)
+        scales.append(s)
+        qh.append(q)
+    for gi in range(sp["g_lo"]):
+        s, q = _quantize_block(C[:, n_hi + gi * GROUP:n_hi + min((gi + 1) * GROUP, n_lo)], 3)
+        scales.append(s)
+        ql.append(q)
+    n = C.shape[0]
+    qh = np.concatenate(qh, axis=1) if qh else np.zeros((n, 0), np.int8)
+    ql = np.concatenate(ql, axis=1) if ql else np.zeros((n, 0), np.int8)
+    return qh, ql, np.stack(scales, axis=1)
+
+
+def dequantize_hadamard_rows(qh, ql, scales, r: int) -> np.ndarray:
+    sp = hadamard_split(r)
+    sh = np.repeat(scales[:, :sp["g_hi"]].astype(np.float64), GROUP, axis=1)[:, :sp["n_hi"]]
+    sl = np.repeat(scales[:, sp["g_hi"]:].astype(np.float64), GROUP, axis=1)[:, :sp["n_lo"]]
+    return np.concatenate([sh * qh, sl * ql], axis=1)
+
+
 def stored_rows(C, r: int, fmt: str) -> np.ndarray:
     """Stored value (fp64) of every row of C (n, r) fp32 in format ``fmt``."""
     if fmt == MIXED:
         return dequantize_rows(*quantize_rows(C, r), r)
+    if fmt == HAD43:
+        return dequantize_hadamard_rows(*quantize_hadamard_rows(C, r), r)
     return store_latents(C, fmt)

@@ -182,3 +182,23 @@ def test_quantize_3bit_group_golden(row):
     assert not qh.any() and not sc[:sp["g_hi"]].view(np.uint16).any()
     assert ql[:len(vals)].tolist() == codes
     assert int(sc[sp["g_hi"]:sp["g_hi"] + 1].view(np.uint16)[0]) == s16_bits
+
+
+def test_vector_quantiser_matches_per_token_definition():
+    g = np.random.default_rng(10)
+    for r in [1, 8, 17, 37, 64, 256, 1000]:
+        C = (g.standard_normal((40, r)) * np.exp(-np.arange(r) / 20)).astype(np.float32)
+        C = (C.astype(np.float64) @ O.hadamard_transform(r)).astype(np.float32)
+        C[3] = 0.0
+        C[5, 0] = 1e7                 # a saturated scale in the first group
+        C[6] *= np.float32(1e-9)      # subnormal (or zero) scales in every group
+        C[7, -1] = 2.5
+        qh, ql, sc = O.quantize_hadamard_rows(C, r)
+        for n in range(C.shape[0]):
+            ah, al, asc = O.quantize_hadamard_latent(C[n], r)
+            assert qh[n].tolist() == ah.tolist()
+            assert ql[n].tolist() == al.tolist()
+            assert sc[n].view(np.uint16).tolist() == asc.view(np.uint16).tolist()
+        want = np.stack([O.dequantize_hadamard_latent(*O.quantize_hadamard_latent(c, r), r) for c in C])
+        np.testing.assert_array_equal(O.dequantize_hadamard_rows(qh, ql, sc, r), want)
+        np.testing.assert_array_equal(O.stored_rows(C, r, O.HAD43), want)
