@@ -1,5 +1,6 @@
 // The C ABI: argument validation, cache layout, launch planning, TMA tensor maps.
 #include <cmath>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -280,6 +281,8 @@ starkv_status starkv_alloc(const starkv_layout* lay, int64_t num_pages, int32_t 
   if (num_pages < 0 || batch < 0 || max_pages < 1 || max_append_tokens < 0)
     return fail(STARKV_ERR_INVALID_ARG, "negative size or max_pages < 1");
   if (max_pages > (1 << 24)) return fail(STARKV_ERR_INVALID_ARG, "max_pages too large");
+  if (static_cast<uint64_t>(num_pages) > SIZE_MAX / static_cast<uint64_t>(lay->page_bytes))
+    return fail(STARKV_ERR_INVALID_ARG, "num_pages * page_bytes does not fit in size_t");
   out->cache_bytes = static_cast<size_t>(num_pages) * lay->page_bytes;
   out->rope_table_bytes = rope_bytes(lay, max_pages);
   out->decode_workspace_bytes = static_cast<size_t>(batch) * lay->cfg.n_q_heads *

@@ -186,3 +186,12 @@ def test_had43_decode_is_refused_before_touching_the_device(lib):
     for name, call in calls.items():
         assert call() == L.ERR_UNSUPPORTED, name
         assert b"had43" in lib.starkv_last_error(), name
+
+
+def test_alloc_rejects_a_cache_size_past_size_t(lib):
+    lay = api.layout_init(api.make_config(32, 8, 128, 4096, 256, [32] * 8, "mixed", 500000.0))
+    s = L.Sizes()
+    huge = (1 << 64) // lay.page_bytes + 1
+    assert huge < (1 << 63)
+    assert lib.starkv_alloc(ctypes.byref(lay), huge, 1, 4, 0, ctypes.byref(s)) == L.ERR_INVALID_ARG
+    assert lib.starkv_alloc(ctypes.byref(lay), huge - 2, 1, 4, 0, ctypes.byref(s)) == L.OK
