@@ -21,6 +21,9 @@ def _ptr(t) -> int | None:
         raise ValueError("expected a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
+    if t.device.index is not None and t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     return t.data_ptr()
 
 

@@ -7,6 +7,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import oracle as O
 from rank_quantized_kv_decode_b200 import _lib as L
@@ -195,3 +196,15 @@ def test_alloc_rejects_a_cache_size_past_size_t(lib):
     assert huge < (1 << 63)
     assert lib.starkv_alloc(ctypes.byref(lay), huge, 1, 4, 0, ctypes.byref(s)) == L.ERR_INVALID_ARG
     assert lib.starkv_alloc(ctypes.byref(lay), huge - 2, 1, 4, 0, ctypes.byref(s)) == L.OK
+
+
+def test_binding_refuses_host_tensors_instead_of_passing_host_pointers(lib):
+    # every device argument goes through the same marshalling; a CPU tensor never reaches the
+    # library as if it were device memory
+    lay = api.layout_init(api.make_config(4, 4, 64, 256, 64, [40, 44, 47, 50], "f32", 10000.0))
+    cpu = torch.zeros(16, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        api.quant_pack(lay, torch.zeros(1, lay.proj_cols), cpu[:1], cpu[:1], cpu[:1].reshape(1, 1),
+                       torch.zeros(lay.page_bytes, dtype=torch.uint8), cpu[:1])
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        api.decode_combine(lay, cpu[:1], 1, torch.zeros(4, 64), torch.zeros(64), torch.zeros(4, 64))
