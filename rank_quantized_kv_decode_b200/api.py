@@ -27,6 +27,51 @@ def _ptr(t) -> int | None:
     return t.data_ptr()
 
 
+def _need(t, name: str, dtype, min_numel: int = 0, ndim: int | None = None) -> None:
+    """Dtype and size a device argument must have, so that the library never reads or writes
+    past the end of a caller's tensor (it sees only a pointer)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dimensions, got shape {tuple(t.shape)}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, at least {min_numel} needed")
+
+
+def _operand_dtype(lay) -> torch.dtype:
+    """dtype of x, A_t and q: fp32 for fp32 latents, else bf16."""
+    return torch.float32 if lay.cfg.fmt == L.FMT["f32"] else torch.bfloat16
+
+
+def _factor_dtype(lay) -> torch.dtype:
+    """dtype of Bk_t: the tensor-core operand type of the format."""
+    f = lay.cfg.fmt
+    return torch.float32 if f == L.FMT["f32"] else (torch.bfloat16 if f == L.FMT["bf16"] else torch.float16)
+
+
+def _check_tokens(n_tok: int, tok_seq, tok_pos, block_table, status) -> None:
+    _need(tok_seq, "tok_seq", torch.int32, n_tok)
+    _need(tok_pos, "tok_pos", torch.int32, n_tok)
+    _need(block_table, "block_table", torch.int32, ndim=2)
+    _need(status, "status", torch.int32, 1)
+
+
+def _check_decode(lay, q, block_table, seq_lens, Bk_t, Bv, out, status) -> None:
+    c = lay.cfg
+    batch = seq_lens.shape[0]
+    _need(seq_lens, "seq_lens", torch.int32, ndim=1)
+    _need(block_table, "block_table", torch.int32, ndim=2)
+    if block_table.shape[0] < batch:
+        raise ValueError(f"block_table: {block_table.shape[0]} rows for {batch} sequences")
+    _need(q, "q", _operand_dtype(lay), batch * c.n_q_heads * c.head_dim)
+    _need(Bk_t, "Bk_t", _factor_dtype(lay), c.n_kv_heads * c.head_dim * c.key_rank)
+    _need(Bv, "Bv", torch.float32, lay.value_rank_total * c.head_dim)
+    _need(out, "out", torch.float32, batch * c.n_q_heads * c.head_dim)
+    _need(status, "status", torch.int32, 1)
+
+
 def _stream(stream) -> int | None:
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream
@@ -69,6 +114,8 @@ def rope_init(lay: L.Layout, max_pages: int, table: torch.Tensor, stream=None) -
 
 def quant_pack(lay, latents, tok_seq, tok_pos, block_table, cache, status, stream=None) -> None:
     n_tok = latents.shape[0]
+    _need(latents, "latents", torch.float32, n_tok * lay.proj_cols)
+    _check_tokens(n_tok, tok_seq, tok_pos, block_table, status)
     L.check(L.load().starkv_quant_pack(
         ctypes.byref(lay), _ptr(latents), n_tok, _ptr(tok_seq), _ptr(tok_pos), _ptr(block_table),
         block_table.shape[1], block_table.shape[0], _ptr(cache),
@@ -78,6 +125,11 @@ def quant_pack(lay, latents, tok_seq, tok_pos, block_table, cache, status, strea
 
 def append(lay, x, A_t, tok_seq, tok_pos, block_table, cache, workspace, status,
            latents_out=None, stream=None) -> None:
+    n_tok = x.shape[0]
+    _need(x, "x", _operand_dtype(lay), n_tok * lay.cfg.d_model)
+    _need(A_t, "A_t", _operand_dtype(lay), lay.proj_cols * lay.cfg.d_model)
+    _need(latents_out, "latents_out", torch.float32, n_tok * lay.proj_cols)
+    _check_tokens(n_tok, tok_seq, tok_pos, block_table, status)
     L.check(L.load().starkv_append(
         ctypes.byref(lay), _ptr(x), x.shape[0], _ptr(A_t), _ptr(tok_seq), _ptr(tok_pos),
         _ptr(block_table), block_table.shape[1], block_table.shape[0], _ptr(cache),
@@ -87,6 +139,9 @@ def append(lay, x, A_t, tok_seq, tok_pos, block_table, cache, workspace, status,
 
 
 def dequant(lay, cache, tok_seq, tok_pos, block_table, latents_out, status, stream=None) -> None:
+    n_tok = tok_seq.shape[0]
+    _need(latents_out, "latents_out", torch.float32, n_tok * lay.proj_cols)
+    _check_tokens(n_tok, tok_seq, tok_pos, block_table, status)
     L.check(L.load().starkv_dequant(
         ctypes.byref(lay), _ptr(cache), cache.numel() * cache.element_size() // lay.page_bytes,
         _ptr(tok_seq), _ptr(tok_pos), tok_seq.shape[0], _ptr(block_table), block_table.shape[1],
@@ -96,6 +151,7 @@ def dequant(lay, cache, tok_seq, tok_pos, block_table, latents_out, status, stre
 def decode_attention(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rope_table, out, workspace,
                      status, max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
                      cta_group: int = 0, stream=None) -> None:
+    _check_decode(lay, q, block_table, seq_lens, Bk_t, Bv, out, status)
     opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms, cta_group)
     L.check(L.load().starkv_decode_attention(
         ctypes.byref(lay), _ptr(q), _ptr(cache),
@@ -111,6 +167,7 @@ def decode_attention_noalloc(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rop
                              stream=None) -> None:
     """decode_attention with the library's built-in 16 MiB scratch instead of a workspace
     (for callers that cannot allocate device memory; see include/starkv.h)."""
+    _check_decode(lay, q, block_table, seq_lens, Bk_t, Bv, out, status)
     opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms, 0)
     L.check(L.load().starkv_decode_attention_noalloc(
         ctypes.byref(lay), _ptr(q), _ptr(cache),
@@ -134,6 +191,7 @@ def decode_plan(lay, batch: int, max_pages: int, max_ctas: int = 0, n_ranges: in
 def decode_partials(lay, q, cache, block_table, seq_lens, Bk_t, rope_table, workspace, status,
                     max_ctas: int = 0, n_ranges: int = 0, timeout_ms: int = 0,
                     cta_group: int = 0, stream=None) -> None:
+    _check_decode(lay, q, block_table, seq_lens, Bk_t, None, None, status)
     opts = L.DecodeOpts(max_ctas, n_ranges, timeout_ms, cta_group)
     L.check(L.load().starkv_decode_partials(
         ctypes.byref(lay), _ptr(q), _ptr(cache),
@@ -145,6 +203,10 @@ def decode_partials(lay, q, cache, block_table, seq_lens, Bk_t, rope_table, work
 
 
 def decode_combine(lay, seq_lens, max_pages: int, Bv, workspace, out, stream=None) -> None:
+    c = lay.cfg
+    _need(seq_lens, "seq_lens", torch.int32, ndim=1)
+    _need(Bv, "Bv", torch.float32, lay.value_rank_total * c.head_dim)
+    _need(out, "out", torch.float32, seq_lens.shape[0] * c.n_q_heads * c.head_dim)
     L.check(L.load().starkv_decode_combine(
         ctypes.byref(lay), _ptr(seq_lens), seq_lens.shape[0], max_pages, _ptr(Bv),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out),
@@ -161,6 +223,13 @@ def absorbed_sizes(lay, batch: int, d_out: int) -> tuple[int, int]:
 
 def absorb_output_weights(lay, Bv, Wo, M, stream=None) -> None:
     """M[rows of head h] = B_v,g(h) Wo[h d:(h+1) d] (fp32, on the device)."""
+    c = lay.cfg
+    _need(Bv, "Bv", torch.float32, lay.value_rank_total * c.head_dim)
+    _need(Wo, "Wo", torch.float32, c.n_q_heads * c.head_dim, ndim=2)
+    if Wo.shape[0] != c.n_q_heads * c.head_dim:
+        raise ValueError(f"Wo: {Wo.shape[0]} rows, expected n_q_heads * head_dim")
+    rows, _ = absorbed_sizes(lay, 1, Wo.shape[1])
+    _need(M, "M", torch.float32, rows * Wo.shape[1])
     L.check(L.load().starkv_absorb_output_weights(ctypes.byref(lay), _ptr(Bv), _ptr(Wo),
                                                   Wo.shape[1], _ptr(M), _stream(stream)),
             "starkv_absorb_output_weights")
@@ -169,6 +238,12 @@ def absorb_output_weights(lay, Bv, Wo, M, stream=None) -> None:
 def decode_combine_absorbed(lay, seq_lens, max_pages: int, M, workspace, scratch, out,
                             stream=None) -> None:
     """Merge the partial records and write out[b] = sum_h a_b,h M_h (out: [batch][d_out])."""
+    _need(seq_lens, "seq_lens", torch.int32, ndim=1)
+    _need(out, "out", torch.float32, ndim=2)
+    if out.shape[0] < seq_lens.shape[0]:
+        raise ValueError(f"out: {out.shape[0]} rows for {seq_lens.shape[0]} sequences")
+    rows, _ = absorbed_sizes(lay, seq_lens.shape[0], out.shape[1])
+    _need(M, "M", torch.float32, rows * out.shape[1])
     L.check(L.load().starkv_decode_combine_absorbed(
         ctypes.byref(lay), _ptr(seq_lens), seq_lens.shape[0], max_pages, _ptr(M), out.shape[1],
         _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(scratch),

@@ -207,4 +207,41 @@ def test_binding_refuses_host_tensors_instead_of_passing_host_pointers(lib):
         api.quant_pack(lay, torch.zeros(1, lay.proj_cols), cpu[:1], cpu[:1], cpu[:1].reshape(1, 1),
                        torch.zeros(lay.page_bytes, dtype=torch.uint8), cpu[:1])
     with pytest.raises(ValueError, match="CUDA tensor"):
-        api.decode_combine(lay, cpu[:1], 1, torch.zeros(4, 64), torch.zeros(64), torch.zeros(4, 64))
+        api.decode_combine(lay, cpu[:1], 1, torch.zeros(lay.value_rank_total, 64), torch.zeros(64),
+                           torch.zeros(4, 64))
+
+
+def test_binding_checks_dtype_and_size_before_the_library_sees_a_pointer(lib):
+    # the library sees only pointers: a tensor of the wrong dtype or too few elements is
+    # refused in the binding (checked before the device check, so this runs on the CPU)
+    lay = api.layout_init(api.make_config(4, 4, 64, 256, 64, [40, 44, 47, 50], "f32", 10000.0))
+    i32 = torch.zeros(4, dtype=torch.int32)
+    table = torch.zeros(2, 4, dtype=torch.int32)
+    cache = torch.zeros(lay.page_bytes, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="latents: expected dtype"):
+        api.quant_pack(lay, torch.zeros(2, lay.proj_cols, dtype=torch.float64), i32, i32, table,
+                       cache, i32)
+    with pytest.raises(ValueError, match="tok_pos: 1 elements"):
+        api.quant_pack(lay, torch.zeros(2, lay.proj_cols), i32, i32[:1], table, cache, i32)
+    with pytest.raises(ValueError, match="block_table: expected 2 dimensions"):
+        api.quant_pack(lay, torch.zeros(2, lay.proj_cols), i32, i32, table.reshape(-1), cache, i32)
+    with pytest.raises(ValueError, match="x: expected dtype"):
+        api.append(lay, torch.zeros(2, 256, dtype=torch.bfloat16),
+                   torch.zeros(lay.proj_cols, 256), i32, i32, table, cache, cache, i32)
+    H, d = 4, 64
+    q = torch.zeros(2, H, d)
+    Bk_t = torch.zeros(4 * d, 64)
+    Bv = torch.zeros(lay.value_rank_total, d)
+    out = torch.zeros(2, H, d)
+    seq_lens = i32[:2]
+    with pytest.raises(ValueError, match="q: 256 elements"):
+        api.decode_attention(lay, q[:1], cache, table, seq_lens, Bk_t, Bv, cache, out, cache, i32)
+    with pytest.raises(ValueError, match="Bk_t: expected dtype"):
+        api.decode_attention(lay, q, cache, table, seq_lens, Bk_t.half(), Bv, cache, out, cache, i32)
+    with pytest.raises(ValueError, match="out: "):
+        api.decode_attention(lay, q, cache, table, seq_lens, Bk_t, Bv, cache, out[:1], cache, i32)
+    with pytest.raises(ValueError, match="block_table: 1 rows for 2 sequences"):
+        api.decode_partials(lay, q, cache, table[:1], seq_lens, Bk_t, cache, cache, i32)
+    # well-formed arguments pass the checks and stop at the device check
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        api.decode_attention(lay, q, cache, table, seq_lens, Bk_t, Bv, cache, out, cache, i32)
