@@ -237,7 +237,9 @@ STARKV_API starkv_status starkv_decode_attention(const starkv_layout* lay, const
 /* Launch shape that starkv_decode_attention / starkv_decode_partials choose for a layout,
  * batch and block-table width on a device with ``num_sms`` SMs and ``smem_per_block`` bytes
  * of opt-in shared memory per block (148 and 232448 on a B200).  Host only, pure: the decode
- * calls make the same choice with the current device's figures. */
+ * calls make the same choice with the current device's figures.  (The pages describe no such
+ * interface; it exposes this library's launch planning.)  INVALID_ARG for a bad layout or
+ * sizes; UNSUPPORTED for a configuration the decode calls would refuse. */
 typedef struct {
   int32_t cta_group;     /* 1: one CTA per 128-token tile; 2: a CTA pair per 256-token tile  */
   int32_t key_mode;      /* int8/int4 keys: 1 = dequantised operand resident per tile, 2 =
