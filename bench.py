@@ -5,9 +5,12 @@
 A step is the whole hot path over one batch: the latent write of the batch's new tokens
 (projection x A, storage into the pages) followed by single-token decode attention over the
 full context (K reconstruction on the tensor cores, RoPE, online softmax, latent P.C_v,
-split combine and up-projection).  Default workload: the Llama-2-7B-shaped MHA layer with
-bf16 latents, batch 8, context 4096.  Metric: KV tokens per second (batch * context / step
-time), with the achieved HBM and tensor-core rates of the dominant kernel beside it.
+split combine and up-projection).  Default workload: the largest stated configuration, the
+Llama-3-8B-shaped GQA layer with int8/int4 latents in 64-token pages, batch 32, context
+32768.  Metric: KV tokens per second (batch * context / step time), with the achieved HBM
+and tensor-core rates of the dominant kernel beside it, and the latent write timed on its
+own (the decode-step append of the batch, and an 8192-token prefill chunk of the long-context
+layer).
 
 With N > 1 (torchrun) every rank runs its own batch of independent sequences (weak
 scaling, no collective on the data path); time is the max over ranks.
@@ -15,6 +18,7 @@ scaling, no collective on the data path); time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -28,13 +32,28 @@ sys.path.insert(0, HERE)
 
 MEASURED_PEAKS = os.path.join(HERE, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# dram bytes per launch of the split kernel from the committed ncu capture of this workload
-# (profiles/decode_split_bf16_llama2_b8_ctx4096.md); set to None when the kernel changes
-SPLIT_TRAFFIC_BYTES = 146703104  # 143.034112 MB read + 3.668992 MB written
+# nominal dense tensor-core rates relative to bf16 (fp16 equals bf16; tf32 is 1.1 of 2.25 PF)
+NOMINAL_RATIO = {"bf16": 1.0, "f16": 1.0, "tf32": 1.1 / 2.25}
+# operand type of the reconstruction MMA per latent format
+MMA_DTYPE = {"f32": "tf32", "bf16": "bf16", "mixed": "f16", "had43": "f16"}
+
+# DRAM bytes (read + write) per launch of the split kernel, from one ncu capture of that
+# workload, keyed by a digest of the kernel's sources: the figure is reported only while the
+# sources are the ones it was captured with (otherwise traffic is null).
+KERNEL_SOURCES = ["decode.cu", "ptx.cuh", "internal.cuh", "api.cu"]
+SPLIT_TRAFFIC = {}  # workload index -> (source digest, bytes)
 
 THROTTLE_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                  0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
                  0x2: "applications_clocks_setting", 0x100: "display_clock_setting"}
+
+
+def kernel_digest() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(HERE, "rank_quantized_kv_decode_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def peaks():
@@ -108,7 +127,7 @@ class OracleDecode:
         from oracle.workloads import ref_for
         import oracle.starkv_oracle as O
         self.O = O
-        self.ref = ref = ref_for(workload_index, False)
+        self.ref = ref = ref_for(workload_index, workload_index in (1, 5))
         self.w = ref.w
         self.q = ref.queries()
         n_seq = max(1, min(n_seq, self.w["batch"]))  # the workload may hold fewer sequences
@@ -183,14 +202,119 @@ def workload_config(w, world):
             "l2": "flushed between steps (256 MiB write outside the timed events)"}
 
 
+def roofline(w, lay, split_ms, pk, src, digest, index):
+    """Roofline of the split kernel (the dominant kernel).  Units: one KV token.  Work per
+    token: 2 r_k H_kv d FLOP of key reconstruction on the tensor cores, and token_bytes of
+    stored latents read from HBM.  The bound is the larger of the two times at their peaks."""
+    B, L = w["batch"], w["context"]
+    tokens = B * L
+    flop = 2.0 * w["key_rank"] * w["n_kv_heads"] * w["head_dim"] * tokens
+    nbytes = float(tokens * lay.token_bytes)
+    dt = MMA_DTYPE[w["fmt"]]
+    peak_tc = pk["bf16_tflops"] * NOMINAL_RATIO[dt]
+    peak_hbm = pk["hbm_gbs"]
+    t_tc = flop / (peak_tc * 1e12)
+    t_hbm = nbytes / (peak_hbm * 1e9)
+    s = split_ms / 1000.0
+    tflops, gbs = flop / s / 1e12, nbytes / s / 1e9
+    traffic = None
+    entry = SPLIT_TRAFFIC.get(index)
+    if entry and entry[0] == digest:
+        traffic = entry[1]
+    common = {"traffic": traffic, "kernel": "decode_split_kernel", "split_ms_median": split_ms,
+              "flop_per_launch": flop, "bytes_per_launch": nbytes,
+              "bound_time_us": max(t_tc, t_hbm) * 1e6,
+              "frac_of_bound_time": max(t_tc, t_hbm) / s,
+              "tensor_achieved_tflops": tflops, "tensor_peak_tflops": peak_tc,
+              "tensor_frac": tflops / peak_tc,
+              "hbm_achieved_gbs": gbs, "hbm_peak_gbs": peak_hbm, "hbm_frac": gbs / peak_hbm,
+              "mma_dtype": dt, "kernel_source_digest": digest,
+              "peak_source": f"{src} ({'bf16 burst' if dt == 'bf16' else f'bf16 burst x nominal {dt}/bf16 ratio'}; HBM copy)"}
+    if t_tc >= t_hbm:
+        return dict({"bound": "tensor", "achieved": tflops, "peak": peak_tc, "unit": "TFLOP/s",
+                     "frac": tflops / peak_tc}, **common)
+    return dict({"bound": "hbm", "achieved": gbs, "peak": peak_hbm, "unit": "GB/s",
+                 "frac": gbs / peak_hbm}, **common)
+
+
+def time_graph(graph, flush, stream, steps, torch):
+    """Median CUDA-event duration (ms) of ``steps`` replays, L2 flushed before each."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        graph.replay()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in evs]))
+
+
+def append_bench(w, lay, pk, steps, dev, torch, api, W, wl, seq, pos, x_new, flush, stream):
+    """The latent write on its own: (1) the decode-step append of this workload's batch (one
+    new token per sequence: projection of B rows, then quantise/pack/scatter), bounded by
+    reading A from HBM; (2) an 8192-token prefill chunk of the long-context GQA layer,
+    bounded by the tensor cores.  Each as tokens/s and as a fraction of its bound."""
+    out = {}
+    launches = 0
+
+    def one(name, lay_, x, A_t, seq_, pos_, table, cache, ws, status):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            api.append(lay_, x, A_t, seq_, pos_, table, cache, ws, status)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        ms = time_graph(g, flush, stream, steps, torch)
+        n = x.shape[0]
+        dm = lay_.cfg.d_model
+        es = x.element_size()
+        flop = 2.0 * n * dm * lay_.proj_cols
+        nbytes = float(lay_.proj_cols * dm * es + n * dm * es + n * lay_.token_bytes)
+        t_tc = flop / (pk["bf16_tflops"] * NOMINAL_RATIO["bf16" if es == 2 else "tf32"] * 1e12)
+        t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+        bound = "tensor" if t_tc >= t_hbm else "hbm"
+        out[name] = {"tokens": n, "us_median": ms * 1000.0, "tokens_per_s": n / (ms / 1000.0),
+                     "bound": bound, "bound_us": max(t_tc, t_hbm) * 1e6,
+                     "frac_of_bound": max(t_tc, t_hbm) / (ms / 1000.0),
+                     "flop": flop, "bytes": nbytes, "kernels": ["project_kernel", "store_kernel"]}
+        return 2 * steps
+
+    launches += one("decode_step", lay, x_new, wl.A_t, seq, pos, wl.block_table, wl.lc.cache,
+                    wl.lc.append_ws, wl.lc.status)
+    # prefill chunk of the long-context layer (its factors; a one-sequence page pool)
+    from rank_quantized_kv_decode_b200 import synth
+    w5 = synth.workload(5)
+    P = w5["prefill_tokens"]
+    st5 = W.setup(dict(w5), need_down=True)
+    cfg5 = api.make_config(w5["n_q_heads"], w5["n_kv_heads"], w5["head_dim"], w5["d_model"],
+                           st5.key_rank, st5.value_ranks, w5["fmt"], w5["rope_theta"])
+    lay5 = api.layout_init(cfg5)
+    mp = P // 64
+    lc5 = api.LatentCache.create(lay5, mp, 1, mp, P, dev)
+    A5 = np.concatenate([st5.Ak] + st5.Av, axis=1)
+    A5_t = torch.from_numpy(np.ascontiguousarray(A5.T, dtype=np.float32)).to(torch.bfloat16).to(dev)
+    x5 = torch.from_numpy(W.hidden_rows(w5, "prefill", P)).to(torch.bfloat16).to(dev)
+    seq5 = torch.zeros(P, dtype=torch.int32, device=dev)
+    pos5 = torch.arange(P, dtype=torch.int32, device=dev)
+    table5 = torch.arange(mp, dtype=torch.int32, device=dev).reshape(1, mp)
+    launches += one("prefill_8192", lay5, x5, A5_t, seq5, pos5, table5, lc5.cache, lc5.append_ws,
+                    lc5.status)
+    torch.cuda.synchronize()
+    assert lc5.status.item() == 0
+    out["prefill_8192"]["workload"] = w5["name"]
+    return out, launches
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-append-bench", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -237,6 +361,7 @@ def main():
         api.decode_combine(lay, wl.seq_lens, lc.max_pages, wl.Bv, lc.decode_ws, wl.out)
 
     calls = (call_append, call_partials, call_combine)
+    launches_per_step = 4  # projection, store, split, combine
     for _ in range(args.warmup):
         flush.fill_(1)
         for c in calls:
@@ -293,8 +418,8 @@ def main():
     # device time of the K steps, max over ranks; every rank processed B sequences
     total_ms = D.max_over_ranks(float(np.sum(step_ms)), dev)
     ms_per_step = total_ms / args.steps
-    tokens_per_step = B * L * world
     value = D.aggregate_rate(B * L * args.steps, world, total_ms / 1000.0)
+    gpu_launches = 2 * launches_per_step * args.steps
 
     # end to end through the public API: host inputs (pinned) in, output back to the host
     x_host = x_new.cpu().pin_memory()
@@ -327,37 +452,31 @@ def main():
     d2h = out_host.numel() * out_host.element_size()
     assert lc.status.item() == 0
 
-    # roofline of the dominant kernel (the split kernel: tensor-core bound reconstruction)
     pk, src = peaks()
-    split_s = float(np.mean(split_ms)) / 1000.0
-    recon_flop = 2.0 * w["key_rank"] * w["n_kv_heads"] * w["head_dim"] * B * L
-    tflops = recon_flop / split_s / 1e12
-    peak_tc = pk["bf16_tflops"]
-    bytes_alg = B * L * lay.token_bytes
-    hbm_gbs = bytes_alg / split_s / 1e9
-    clk = clocks.summary()
+    rl = roofline(w, lay, float(np.median(split_ms)), pk, src, kernel_digest(), args.workload)
     line = {
         "metric": "compressed-KV decode attention KV tokens/s", "value": value,
         "unit": "KV tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if w["fmt"] == "bf16" else w["fmt"],
+        "ms_per_step": ms_per_step, "ms_per_step_median": float(np.median(step_ms)),
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {"bf16": "bf16", "f32": "f32"}.get(w["fmt"], "int8/int4+f16"),
         "data": "synthetic (seeded latents with the stated singular-value spectra)",
         "config": workload_config(w, world),
-        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tc, "unit": "TFLOP/s",
-                     "frac": tflops / peak_tc, "traffic": SPLIT_TRAFFIC_BYTES,
-                     "peak_source": f"{src} bf16 burst", "kernel": "decode_split_kernel",
-                     "peak_sustained": pk.get("bf16_tflops_sustained"),
-                     "frac_of_sustained": (tflops / pk["bf16_tflops_sustained"]
-                                           if pk.get("bf16_tflops_sustained") else None),
-                     "flop_per_launch": recon_flop, "split_ms": split_s * 1000.0,
-                     "hbm_achieved_gbs": hbm_gbs, "hbm_peak_gbs": pk["hbm_gbs"],
-                     "hbm_frac": hbm_gbs / pk["hbm_gbs"], "hbm_bytes_per_launch": bytes_alg},
+        "roofline": rl,
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        # pass 1: append (projection + store), split, combine per step; pass 2: the same
-        "gpu_launches": 8 * args.steps,
-        "clocks": clk,
+        "clocks": clocks.summary(),
     }
+    e2e_launches = launches_per_step * args.steps
+    if not args.no_append_bench:
+        with ClockSampler(local) as aclk:
+            app, n = append_bench(w, lay, pk, args.steps, dev, torch, api, W, wl, seq, pos, x_new,
+                                  flush, stream)
+        app["clocks"] = aclk.summary()
+        line["append"] = app
+        gpu_launches += n
+    line["gpu_launches"] = gpu_launches
+    line["gpu_launches_e2e"] = e2e_launches
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, dt, cores, sample = cpu_baseline(args.workload)
         line["cpu_baseline"] = {"value": v, "unit": "KV tokens/s", "cores": cores, "kind": "oracle",

@@ -326,11 +326,16 @@ STARKV_API starkv_status starkv_decode_combine_absorbed(
  *     GPU that loads the library holds it until the process exits.  Calls whose records need
  *     more (batch * n_q_heads * ceil(max_pages / 2) * 4 * ceil((2 + value_rank_max) / 4)
  *     floats) return STARKV_ERR_WORKSPACE with a message; nothing is launched.
- *   - The first call on a device looks up the array's device address (once per device, with
- *     that device current); make that first call before any stream capture.
+ *   - The first call in a CUDA context (the device's primary context, or a context the
+ *     caller made current) looks up the array's device address in that context and keeps
+ *     it, keyed on the context's unique ID; a context created again after cudaDeviceReset
+ *     gets a fresh lookup.  Make that first call before any stream capture.
  *   - All calls share the array and it keeps the last call's contents.  Nothing in it needs
  *     to start at zero: each call writes every record it reads.  Calls whose kernels overlap
- *     on the GPU (two streams, two threads, two graphs) race on it.
+ *     on the GPU (two streams, two threads, two graphs) race on it.  A CUDA graph that
+ *     captured this call holds the array's address, so every such graph shares the one
+ *     array too: replays of two of them must be ordered on the GPU, and the device status
+ *     word does not show a race.
  *   - Allocates nothing (no cudaMalloc / cudaFree).  Other arguments, results and errors as
  *     starkv_decode_attention. */
 STARKV_API starkv_status starkv_decode_attention_noalloc(

@@ -601,6 +601,40 @@ def latent_attention(q, C_k, C_v, B_k, theta: float, n_kv_heads: int, heads=None
     return out
 
 
+def tile_partials(q, C_k, C_v, B_k, theta: float, n_kv_heads: int, tile: int = 128, heads=None):
+    """The split-K view of latent_attention: per query head h and per block of ``tile``
+    consecutive positions [t0, t0 + tile), the block's largest score in log2 units
+    m = max_t s_t log2(e), its weight sum l = sum_t 2^(s_t log2(e) - m) and its unnormalised
+    latent sum a = sum_t 2^(s_t log2(e) - m) c_v,g(h),t, with s_t = q'.k'_t/sqrt(d) as in
+    latent_attention.  The exact merge of the blocks (log-sum-exp) is latent_attention's a_h:
+    a_h = sum_b 2^(m_b - M) a_b / sum_b 2^(m_b - M) l_b, M = max_b m_b.
+    Returns, for each head of ``heads`` (default all), a list over blocks of (m, l, a)."""
+    q = np.asarray(q, dtype=np.float64)
+    H, d = q.shape
+    G = H // n_kv_heads
+    L = C_k.shape[0]
+    heads = range(H) if heads is None else heads
+    pos = np.arange(L)
+    log2e = 1.0 / math.log(2.0)
+    out = []
+    cache_k = {}
+    for h in heads:
+        g = h // G
+        if g not in cache_k:
+            Bg = np.asarray(B_k, np.float64)[:, g * d:(g + 1) * d]
+            cache_k[g] = apply_rope(np.asarray(C_k, np.float64) @ Bg, pos, theta)
+        s = cache_k[g] @ apply_rope(q[h], L - 1, theta) / math.sqrt(d) * log2e
+        Cv = np.asarray(C_v[g], np.float64)
+        blocks = []
+        for t0 in range(0, L, tile):
+            sb = s[t0:t0 + tile]
+            m = sb.max()
+            w = np.power(2.0, sb - m)
+            blocks.append((m, w.sum(), w @ Cv[t0:t0 + tile]))
+        out.append(blocks)
+    return out
+
+
 def decode_attention(q, C_k, C_v, B_k, B_v, theta: float, n_kv_heads: int, heads=None):
     """Single-token decode attention of one sequence from its stored latents: the latent
     outputs a_h of latent_attention, up-projected o_h = a_h B_v,g(h) (B_v: list over g of

@@ -158,6 +158,26 @@ size_t rope_bytes(const starkv_layout* lay, int max_pages) {
 int record_floats(const starkv_layout* lay) { return (2 + lay->value_rank_max + 3) / 4 * 4; }
 int tiles_for(int max_pages) { return ceil_div(max_pages * kPage, kTile); }
 
+// Bytes of the decode partial records of `batch` sequences: batch * n_q_heads * tiles * rec
+// floats, multiplied in 64 bits with an overflow check at every step.  Also refuses a
+// batch * n_q_heads above the combine kernel's grid limit (one CTA per sequence and head).
+starkv_status decode_ws_bytes(const starkv_layout* lay, int32_t batch, int32_t max_pages,
+                              size_t* out) {
+  const uint64_t factors[4] = {static_cast<uint64_t>(lay->cfg.n_q_heads),
+                               static_cast<uint64_t>(tiles_for(max_pages)),
+                               static_cast<uint64_t>(record_floats(lay)), sizeof(float)};
+  if (static_cast<uint64_t>(batch) * factors[0] > 0x7FFFFFFFull)
+    return fail(STARKV_ERR_INVALID_ARG, "batch * n_q_heads above 2^31 - 1");
+  uint64_t n = static_cast<uint64_t>(batch);
+  for (uint64_t f : factors) {
+    if (f != 0 && n > SIZE_MAX / f)
+      return fail(STARKV_ERR_INVALID_ARG, "decode workspace size does not fit in size_t");
+    n *= f;
+  }
+  *out = static_cast<size_t>(n);
+  return STARKV_OK;
+}
+
 void fill_store(StoreParams& sp, const starkv_layout* lay) {
   sp.fmt = lay->cfg.fmt;
   sp.n_lat = lay->n_latents;
@@ -285,8 +305,8 @@ starkv_status starkv_alloc(const starkv_layout* lay, int64_t num_pages, int32_t 
     return fail(STARKV_ERR_INVALID_ARG, "num_pages * page_bytes does not fit in size_t");
   out->cache_bytes = static_cast<size_t>(num_pages) * lay->page_bytes;
   out->rope_table_bytes = rope_bytes(lay, max_pages);
-  out->decode_workspace_bytes = static_cast<size_t>(batch) * lay->cfg.n_q_heads *
-                                tiles_for(max_pages) * record_floats(lay) * sizeof(float);
+  st = decode_ws_bytes(lay, batch, max_pages, &out->decode_workspace_bytes);
+  if (st != STARKV_OK) return st;
   size_t ws = 0;
   for (int m = 1; m <= ceil_div(max_append_tokens, 128); ++m) {
     const int n = std::min(max_append_tokens, 128 * m);
@@ -648,9 +668,9 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   if (split && rope_table_bytes < rope_bytes(lay, max_pages))
     return fail(STARKV_ERR_WORKSPACE, "rope table smaller than needed for max_pages");
   const starkv_config& c = lay->cfg;
-  const int tiles_max = tiles_for(max_pages);
-  const int rec = record_floats(lay);
-  const size_t ws_need = static_cast<size_t>(batch) * c.n_q_heads * tiles_max * rec * sizeof(float);
+  size_t ws_need = 0;
+  st = decode_ws_bytes(lay, batch, max_pages, &ws_need);
+  if (st != STARKV_OK) return st;
   if (workspace_bytes < ws_need) return fail(STARKV_ERR_WORKSPACE, "decode workspace too small");
   DevInfo info;
   st = current_device(info);

@@ -20,34 +20,103 @@ constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-// Device address of g_decode_scratch, looked up once per device (with that device current).
-// Host code may not pass the symbol itself to a kernel: on the host it is only a stand-in.
-std::mutex g_mu;
-void* g_scratch_ptr[64] = {};
+// Device address of g_decode_scratch.  The address belongs to the CUDA context that loaded
+// the library's module, so it is cached per context, keyed on the context's unique ID (a
+// context that is destroyed and created again, e.g. after cudaDeviceReset, gets a new ID, and
+// a caller's own non-primary context gets its own entry).  Host code may not pass the symbol
+// itself to a kernel: on the host it is only a stand-in.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-starkv_status scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    starkv::set_error_message(std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+
+std::mutex g_mu;
+ScratchEntry g_scratch[64] = {};
+int g_scratch_n = 0, g_scratch_next = 0;
+
+starkv_status driver_fns(CtxGetCurrentFn& get_current, CtxGetIdFn& get_id) {
+  static std::once_flag once;
+  static CtxGetCurrentFn s_current = nullptr;
+  static CtxGetIdFn s_id = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      s_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      s_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!s_current || !s_id) {
+    starkv::set_error_message("cuCtxGetCurrent / cuCtxGetId not available from the driver");
     return STARKV_ERR_CUDA;
   }
-  if (dev < 0 || dev >= 64) {
-    starkv::set_error_message("device index above 63");
-    return STARKV_ERR_UNSUPPORTED;
+  get_current = s_current;
+  get_id = s_id;
+  return STARKV_OK;
+}
+
+starkv_status symbol_address(void** p) {
+  *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(p, g_decode_scratch);
+  if (e != cudaSuccess || *p == nullptr) {
+    starkv::set_error_message(std::string("cudaGetSymbolAddress(decode scratch): ") +
+                              cudaGetErrorString(e));
+    return STARKV_ERR_CUDA;
+  }
+  return STARKV_OK;
+}
+
+starkv_status scratch_address(void** out) {
+  CtxGetCurrentFn get_current;
+  CtxGetIdFn get_id;
+  starkv_status st = driver_fns(get_current, get_id);
+  if (st != STARKV_OK) return st;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) {
+    starkv::set_error_message("cuCtxGetCurrent failed");
+    return STARKV_ERR_CUDA;
   }
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      starkv::set_error_message(std::string("cudaGetSymbolAddress(decode scratch): ") +
-                                cudaGetErrorString(e));
+  void* p = nullptr;
+  if (ctx == nullptr) {
+    // no context yet on this thread: the lookup itself makes the device's primary context
+    // current (the runtime's rule), then its ID keys the entry
+    st = symbol_address(&p);
+    if (st != STARKV_OK) return st;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
+      starkv::set_error_message("no current CUDA context after the symbol lookup");
       return STARKV_ERR_CUDA;
     }
-    g_scratch_ptr[dev] = p;
   }
-  *out = g_scratch_ptr[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) {
+    starkv::set_error_message("cuCtxGetId failed");
+    return STARKV_ERR_CUDA;
+  }
+  for (int i = 0; i < g_scratch_n; ++i) {
+    if (g_scratch[i].ctx_id == id) {
+      *out = g_scratch[i].ptr;
+      return STARKV_OK;
+    }
+  }
+  if (p == nullptr) {
+    st = symbol_address(&p);
+    if (st != STARKV_OK) return st;
+  }
+  // a small ring of contexts: an entry of a context that no longer exists is only ever
+  // overwritten, never used (context IDs are not reused within a process)
+  ScratchEntry& slot = g_scratch[g_scratch_next];
+  slot.ctx_id = id;
+  slot.ptr = p;
+  g_scratch_next = (g_scratch_next + 1) % 64;
+  if (g_scratch_n < 64) ++g_scratch_n;
+  *out = p;
   return STARKV_OK;
 }
 

@@ -198,6 +198,29 @@ def test_alloc_rejects_a_cache_size_past_size_t(lib):
     assert lib.starkv_alloc(ctypes.byref(lay), huge - 2, 1, 4, 0, ctypes.byref(s)) == L.OK
 
 
+def test_decode_workspace_size_is_checked_for_overflow(lib):
+    """batch * n_q_heads * tiles * record floats * 4 must not wrap: a wrapped size could pass
+    both the caller-workspace check and the no-allocation entry point's scratch check."""
+    lay = api.layout_init(api.make_config(512, 64, 128, 4096, 256, [128] * 64, "mixed", 1e4))
+    s = L.Sizes()
+    # 2^31 - 1 sequences x 512 heads: above the combine's grid limit (and past 2^64 bytes)
+    assert lib.starkv_alloc(ctypes.byref(lay), 1, (1 << 31) - 1, 1 << 24, 0,
+                            ctypes.byref(s)) == L.ERR_INVALID_ARG
+    assert b"2^31" in lib.starkv_last_error()
+    # the largest batch the grid allows: the size is exact (below 2^64, no wrap)
+    b = ((1 << 31) - 1) // 512
+    assert lib.starkv_alloc(ctypes.byref(lay), 1, b, 1 << 24, 0, ctypes.byref(s)) == L.OK
+    assert s.decode_workspace_bytes == b * 512 * (1 << 23) * 132 * 4
+    # and the no-allocation entry point refuses the oversized batch before touching a device
+    rc = lib.starkv_decode_attention_noalloc(
+        ctypes.byref(lay), None, None, 1, None, 1 << 24, None, (1 << 31) - 1, None, None, None,
+        0, None, None, None, None)
+    assert rc == L.ERR_INVALID_ARG
+    # an ordinary size is exact
+    assert lib.starkv_alloc(ctypes.byref(lay), 1, 3, 10, 0, ctypes.byref(s)) == L.OK
+    assert s.decode_workspace_bytes == 3 * 512 * 5 * (4 * ((2 + 128 + 3) // 4)) * 4
+
+
 def test_binding_refuses_host_tensors_instead_of_passing_host_pointers(lib):
     # every device argument goes through the same marshalling; a CPU tensor never reaches the
     # library as if it were device memory

@@ -14,7 +14,7 @@ from oracle.workloads import ref_for
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("index,n_tok", [(1, 300), (5, 8), (5, 333), (2, 8)])
+@pytest.mark.parametrize("index,n_tok", [(1, 300), (5, 8), (5, 333), (2, 8), (3, 16), (3, 200), (4, 32)])
 def test_append_projection_and_store(index, n_tok):
     ref = ref_for(index, True)
     w = ref.w

@@ -158,3 +158,52 @@ def test_single_token_context():
     Bv = [g.standard_normal((3, 16))]
     out = O.decode_attention(g.standard_normal((2, 16)), Ck, Cv, Bk, Bv, 10000.0, 1)
     np.testing.assert_allclose(out, np.stack([Cv[0][0] @ Bv[0]] * 2), rtol=1e-12)
+
+
+def _tiny_latents(seed, L, H, Hkv, d, rk, ranks):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((H, d))
+    Ck = g.standard_normal((L, rk))
+    Cv = [g.standard_normal((L, r)) for r in ranks]
+    Bk = g.standard_normal((rk, Hkv * d)) / math.sqrt(rk)
+    return q, Ck, Cv, Bk
+
+
+@pytest.mark.parametrize("L,tile", [(1, 128), (5, 2), (300, 128), (256, 128), (7, 7)])
+def test_tile_partials_merge_to_latent_attention(L, tile):
+    """The log-sum-exp merge of the per-block records is the whole-sequence softmax output."""
+    H, Hkv, d = 4, 2, 8
+    q, Ck, Cv, Bk = _tiny_latents(L, L, H, Hkv, d, 6, [3, 5])
+    want = O.latent_attention(q, Ck, Cv, Bk, 10000.0, Hkv)
+    parts = O.tile_partials(q, Ck, Cv, Bk, 10000.0, Hkv, tile=tile)
+    for h in range(H):
+        blocks = parts[h]
+        assert len(blocks) == -(-L // tile)
+        M = max(m for m, _, _ in blocks)
+        num = sum(2.0 ** (m - M) * a for m, _, a in blocks)
+        den = sum(2.0 ** (m - M) * l for m, l, _ in blocks)
+        np.testing.assert_allclose(num / den, want[h], rtol=1e-12, atol=1e-14)
+        for m, l, a in blocks:
+            # the block's own maximum term is 2^0 = 1: 1 <= l <= block length
+            assert 1.0 - 1e-12 <= l <= tile + 1e-12
+
+
+def test_tile_partials_hand_worked():
+    """d = 2 (one RoPE pair, frequency 1), one KV head, keys reconstructed by an identity B:
+    the scores are q'.k'_t / sqrt(2) with q' rotated by (L-1) and k_t by t radians."""
+    q = np.array([[1.0, 0.0]])
+    Ck = np.array([[1.0, 0.0], [0.0, 1.0], [2.0, 0.0]])  # L = 3
+    Cv = [np.array([[1.0], [10.0], [100.0]])]
+    Bk = np.eye(2)
+    parts = O.tile_partials(q, Ck, Cv, Bk, 10000.0, 1, tile=2)
+    # q' = (cos 2, sin 2); k'_0 = (1, 0); k'_1 = rot(1)(0, 1) = (-sin 1, cos 1);
+    # k'_2 = rot(2)(2, 0) = (2 cos 2, 2 sin 2)
+    s = np.array([math.cos(2),
+                  -math.cos(2) * math.sin(1) + math.sin(2) * math.cos(1),
+                  2.0]) / math.sqrt(2) / math.log(2)
+    (m0, l0, a0), (m1, l1, a1) = parts[0]
+    assert m0 == pytest.approx(max(s[0], s[1]), abs=1e-14)
+    assert l0 == pytest.approx(2 ** (s[0] - m0) + 2 ** (s[1] - m0), abs=1e-14)
+    assert a0[0] == pytest.approx(2 ** (s[0] - m0) * 1 + 2 ** (s[1] - m0) * 10, abs=1e-12)
+    assert (m1, l1) == (pytest.approx(s[2], abs=1e-14), pytest.approx(1.0, abs=1e-15))
+    assert a1[0] == pytest.approx(100.0, abs=1e-12)
