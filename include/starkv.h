@@ -78,9 +78,8 @@ typedef enum {
   STARKV_FMT_HAD43 = 3  /* STAR-KV technical summary, Methodology §3: latents of factors
                            rotated by a block-wise Hadamard transform, the leading
                            ceil(r/5) channels as 4-bit codes, the rest as 3-bit codes, fp16
-                           group scales.  Layout, store (starkv_quant_pack, starkv_append:
-                           bf16 operands) and read-back so far; the decode calls return
-                           STARKV_ERR_UNSUPPORTED */
+                           group scales; fp16 tensor cores.  The caller folds the rotation
+                           into the factors (A T, T^T B); append takes bf16 operands */
 } starkv_fmt;
 
 /* Model/cache description (host struct, POD). */
@@ -214,7 +213,7 @@ STARKV_API starkv_status starkv_dequant(const starkv_layout* lay, const void* ca
  *              bf16 (fmt bf16/mixed) or fp32 (fmt f32)
  *   seq_lens   device int32 [batch]; 0 gives a zero output row
  *   Bk_t       device [H_kv*d][key_rank], row n = column n of B_k: fp32 (f32), bf16 (bf16),
- *              fp16 (mixed) -- the tensor-core operand type of the format
+ *              fp16 (mixed, had43) -- the tensor-core operand type of the format
  *   Bv         device fp32 [value_rank_total][d]: B_v,g stacked in head order (rows
  *              seg[1+g].col - key_rank ...)
  *   rope_table device, from starkv_rope_init with max_pages >= this call's max_pages

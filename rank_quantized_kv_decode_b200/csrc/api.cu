@@ -125,12 +125,14 @@ starkv_status check_layout(const starkv_layout* lay) {
   return STARKV_OK;
 }
 
-// The formats the decode kernels implement (had43 has its store and read-back only).
+// The formats the decode kernels implement: all four (f32, bf16, int8/int4, had43).
 starkv_status check_decode_format(const starkv_layout* lay) {
-  if (lay->cfg.fmt == STARKV_FMT_HAD43)
-    return fail(STARKV_ERR_UNSUPPORTED, "decode of the had43 format is not implemented yet");
+  (void)lay;
   return STARKV_OK;
 }
+
+// Formats stored as codes with fp16 group scales, decoded by the dequantisers.
+bool quantised(int fmt) { return fmt == STARKV_FMT_MIXED || fmt == STARKV_FMT_HAD43; }
 
 // Split-K plan of the projection: about one CTA per SM of a B200 (148), every split non-empty.
 constexpr int kProjCtaTarget = 148;
@@ -506,7 +508,7 @@ static starkv_status plan_shape(const starkv_layout* lay, int32_t batch, int32_t
   // the streamed int8/int4 operand (key rank > 256, dequantised per ring stage) ran slower on
   // pairs than on single CTAs (10.1 vs 12.0 ms at batch 16, context 16384, rank 1024): the
   // default keeps single-CTA tiles there
-  const bool pair_default = pair_ok && !(fmt == STARKV_FMT_MIXED && p.kb_count > 4);
+  const bool pair_default = pair_ok && !(quantised(fmt) && p.kb_count > 4);
   p.cta_group = want_cg == 2 ? 2 : (want_cg == 1 ? 1 : (pair_default ? 2 : 1));
   const int CG = p.cta_group;
   int grid_cap = sms;
@@ -538,7 +540,7 @@ static starkv_status plan_shape(const starkv_layout* lay, int32_t batch, int32_t
     const starkv_segment& first = lay->seg[1 + g0];
     const starkv_segment& last = lay->seg[g1];
     int64_t start, end;
-    if (fmt == STARKV_FMT_MIXED) {
+    if (quantised(fmt)) {
       start = first.off_i8;
       end = last.off_sc + static_cast<int64_t>(kPage) * 2 * (last.g8 + last.g4);
     } else {
@@ -558,7 +560,7 @@ static starkv_status plan_shape(const starkv_layout* lay, int32_t batch, int32_t
   // fit, else the dequantisers read the codes from global memory (mode 0)
   int modes[2] = {0, 0};
   int n_modes = 1;
-  if (fmt == STARKV_FMT_MIXED) {
+  if (quantised(fmt)) {
     if (p.kb_count <= 4) {
       modes[0] = 1;
     } else {
@@ -570,7 +572,7 @@ static starkv_status plan_shape(const starkv_layout* lay, int32_t batch, int32_t
   int key_region = 0;
   {
     const starkv_segment& k = lay->seg[0];
-    if (fmt == STARKV_FMT_MIXED)
+    if (quantised(fmt))
       key_region = static_cast<int>(k.off_sc + int64_t(kPage) * 2 * (k.g8 + k.g4) - k.off_i8);
   }
   // shared-memory plan: ring stages of (A k-block, B k-block), value buffers, small arrays
@@ -694,7 +696,7 @@ static starkv_status plan_decode(const starkv_layout* lay, const void* q, const 
   std::memset(&tmB, 0, sizeof(tmB));
   if (!split) return STARKV_OK;
   const cuuint32_t ke = static_cast<cuuint32_t>(kKBytes / es);
-  if (fmt != STARKV_FMT_MIXED) {
+  if (!quantised(fmt)) {
     const CUtensorMapDataType dt =
         fmt == STARKV_FMT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(c.key_rank), static_cast<cuuint64_t>(kPage),

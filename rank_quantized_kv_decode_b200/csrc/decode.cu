@@ -32,6 +32,9 @@ namespace {
 constexpr int FMT_F32 = STARKV_FMT_F32;
 constexpr int FMT_BF16 = STARKV_FMT_BF16;
 constexpr int FMT_MIXED = STARKV_FMT_MIXED;
+// the pages' own 4-bit/3-bit block-Hadamard format: decoded by the int8/int4 machinery (staged
+// codes, fp16 operand) with its own code layout
+constexpr int FMT_HAD43 = STARKV_FMT_HAD43;
 
 struct Unit {
   int b, tile, c0, c1, L, nvalid;
@@ -91,7 +94,8 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
 
 template <int FMT>
 struct Fmt {
-  static constexpr bool kTmaA = FMT != FMT_MIXED;
+  static constexpr bool kQuant = FMT == FMT_MIXED || FMT == FMT_HAD43;  // codes + fp16 scales
+  static constexpr bool kTmaA = !kQuant;
   // fp32 operands: 3xTF32 (hi*hi + hi*lo + lo*hi), the hi/lo split done in shared memory
   static constexpr bool kSplit = FMT == FMT_F32;
   static constexpr int kKind = FMT == FMT_F32 ? 1 : 0;
@@ -107,7 +111,9 @@ struct Fmt {
 struct VChan {
   int off, stride;
   int soff, sstride;
-  int lsh, rsh;  // signed code = (byte << lsh) >> rsh: int8 (24, 24), low / high nibble (28 / 24, 28)
+  int lsh, rsh;  // signed code = (w << lsh) >> rsh: int8 (24, 24), low / high nibble (28 / 24, 28),
+                 // 3-bit field at bit b of a little-endian byte pair (29 - b, 29)
+  int two;       // had43 3-bit channel: the code's bits may reach into the next byte
 };
 
 template <int FMT>
@@ -119,6 +125,19 @@ __device__ __forceinline__ VChan vchan(const LatDesc& vd, int vbase, int i) {
   } else if constexpr (FMT == FMT_BF16) {
     v.off = vd.off0 - vbase + 2 * i;
     v.stride = 2 * vd.rank;
+  } else if constexpr (FMT == FMT_HAD43) {
+    // 4-bit channels [0, n8) two per byte (pitch bytes per token); 3-bit channels eight per
+    // 3-byte word, code j at bits [3 (j mod 8), +3) of word j / 8 (nb4 bytes per token)
+    const bool hi = i < vd.n8;
+    const int j = i - vd.n8;
+    const int bit = 3 * (j & 7);
+    v.off = hi ? vd.off0 - vbase + (i >> 1) : vd.off1 - vbase + 3 * (j >> 3) + (bit >> 3);
+    v.stride = hi ? vd.pitch : vd.nb4;
+    v.lsh = hi ? ((i & 1) ? 24 : 28) : 29 - (bit & 7);
+    v.rsh = hi ? 28 : 29;
+    v.two = hi ? 0 : ((bit & 7) > 5);
+    v.soff = vd.off2 - vbase + 2 * (hi ? (i >> 5) : vd.g8 + (j >> 5));
+    v.sstride = 2 * vd.ng;
   } else {
     const bool is8 = i < vd.n8;
     const int j = i - vd.n8;
@@ -139,7 +158,10 @@ __device__ __forceinline__ float vchan_load(const uint8_t* slot, const VChan& v,
   } else if constexpr (FMT == FMT_BF16) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(slot + v.off + row * v.stride));
   } else {
-    const unsigned b = slot[v.off + row * v.stride];
+    unsigned b = slot[v.off + row * v.stride];
+    if constexpr (FMT == FMT_HAD43) {
+      if (v.two) b |= static_cast<unsigned>(slot[v.off + 1 + row * v.stride]) << 8;
+    }
     const int q = static_cast<int>(b << v.lsh) >> v.rsh;
     const float s = __half2float(*reinterpret_cast<const __half*>(slot + v.soff + row * v.sstride));
     // q as a float without the conversion unit: 1.5 * 2^23 + q has an ulp of 1, so its bits
@@ -170,11 +192,26 @@ __device__ __forceinline__ void load_p(const float* ptr, float (&out)[G]) {
   }
 }
 
-// 8 consecutive key-latent channels [k0, k0+8) of one token as fp16 (scale * code, rounded
-// to nearest), packed for one 16-byte store.  ``base`` is the page.
+// Key-latent channel k of token row ``prow`` as the exact fp32 product scale * code.  ``base``
+// is the page (or a copy of its key blocks with the offsets rebased).
+template <bool H43>
 __device__ __forceinline__ float key_code_value(const uint8_t* base, const LatDesc& kd, int prow,
                                                 int k) {
   const __half* sc = reinterpret_cast<const __half*>(base + kd.off2) + prow * kd.ng;
+  if constexpr (H43) {
+    if (k < kd.n8) {  // 4-bit: two codes per byte
+      const uint8_t byte = (base + kd.off0)[prow * kd.pitch + (k >> 1)];
+      const int nib = (k & 1) ? (byte >> 4) : (byte & 15);
+      return __half2float(sc[k >> 5]) * static_cast<float>((nib ^ 8) - 8);
+    }
+    // 3-bit: code j at bits [3 (j mod 8), +3) of the 3-byte word j / 8
+    const int j = k - kd.n8;
+    const int bit = 3 * (j & 7);
+    const uint8_t* w = base + kd.off1 + prow * kd.nb4 + 3 * (j >> 3) + (bit >> 3);
+    const unsigned pair = w[0] | (static_cast<unsigned>(w[1]) << 8);
+    const int f = static_cast<int>((pair >> (bit & 7)) & 7u);
+    return __half2float(sc[kd.g8 + (j >> 5)]) * static_cast<float>((f ^ 4) - 4);
+  }
   if (k < kd.n8) {
     const int8_t q = reinterpret_cast<const int8_t*>(base + kd.off0)[prow * kd.n8 + k];
     return __half2float(sc[k >> 5]) * static_cast<float>(q);
@@ -204,12 +241,13 @@ __device__ __forceinline__ uint32_t h2_bits(__half2 h) {
 // offsets of ``kd`` (the page itself in global memory, or a copy of its key region in shared
 // memory with the offsets rebased), one channel at a time: the ragged edges of the int8 and
 // int4 parts.
+template <bool H43>
 __device__ __forceinline__ uint4 dequant8_at(const uint8_t* base, const LatDesc& kd, int prow, int k0) {
   float v[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const int k = k0 + e;
-    v[e] = k < kd.rank ? key_code_value(base, kd, prow, k) : 0.f;
+    v[e] = k < kd.rank ? key_code_value<H43>(base, kd, prow, k) : 0.f;
   }
   return make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]),
                     pack_h2(v[6], v[7]));
@@ -223,11 +261,111 @@ __device__ __forceinline__ uint4 dequant8_at(const uint8_t* base, const LatDesc&
 // memory, so the compiler could not move a later row's load above an earlier row's store.
 constexpr uint32_t kNoRow = 0xFFFFFFFFu;
 
+// The 32-bit word of the codes at byte address ``a`` (any alignment), from the two aligned words
+// that cover it; the bytes past the codes lie inside the page's blocks (the next block or the
+// scales follow every code block).
+template <bool SMEM>
+__device__ __forceinline__ uint32_t word_at(uint32_t a_smem, const uint8_t* a_glob) {
+  if constexpr (SMEM) {
+    const uint32_t al = a_smem & ~3u;
+    return __funnelshift_r(ld_shared_u32(al), ld_shared_u32(al + 4), (a_smem & 3u) * 8u);
+  } else {
+    const uintptr_t ga = reinterpret_cast<uintptr_t>(a_glob);
+    const uint32_t* al = reinterpret_cast<const uint32_t*>(ga & ~static_cast<uintptr_t>(3));
+    return __funnelshift_r(al[0], al[1], static_cast<uint32_t>(ga & 3u) * 8u);
+  }
+}
+
+// had43 key channels [k0, k0+8) of 8 tile rows, as dequant_rows8 (below) does for int8/int4:
+// inside the 4-bit block, nibbles as int4 codes (bias 8); inside the 3-bit block, the 8 codes
+// of the group from a 48-bit window (their first code need not start a 3-byte word), each pair
+// as exact fp16 under the exponent bits of 1024 with bias 4, times its group's fp16 scale
+// (a group of 8 may straddle two 32-channel scale groups).  Returns false when the group
+// straddles the 4-bit/3-bit boundary or the end of the latent (the caller's per-channel path).
 template <bool SMEM, class BaseFn>
+__device__ __forceinline__ bool dequant_rows8_h43(uint32_t dst, const LatDesc& kd, int k0, int ch,
+                                                  int row0, BaseFn key_base, uint32_t safe) {
+  const bool b4 = k0 + 8 <= kd.n8;
+  const bool b3 = k0 >= kd.n8 && k0 + 8 <= kd.rank;
+  if (!b4 && !b3) return false;
+  const int j0 = k0 - kd.n8;
+  const int sg0 = b4 ? (k0 >> 5) : kd.g8 + (j0 >> 5);  // scale group of the first code
+  const int split = b4 ? 8 : min(8, 32 - (j0 & 31));      // codes before the next group
+#pragma unroll 2
+  for (int it = 0; it < 8; ++it) {
+    const int r = row0 + 16 * it;
+    const int prow = r & 63;
+    const auto b = key_base(it, r);
+    bool ok;
+    uint32_t w0 = 0, w1 = 0;
+    unsigned short s0 = 0, s1 = 0;
+    if constexpr (SMEM) {
+      ok = b != kNoRow;
+      const uint32_t bs = ok ? b : safe;
+      const uint32_t sa = bs + kd.off2 + 2 * (prow * kd.ng + sg0);
+      s0 = ld_shared_u16(sa);
+      s1 = split < 8 ? ld_shared_u16(sa + 2) : s0;
+      if (b4) {
+        w0 = word_at<true>(bs + kd.off0 + prow * kd.pitch + (k0 >> 1), nullptr);
+      } else {
+        const uint32_t a = bs + kd.off1 + prow * kd.nb4 + 3 * (j0 >> 3);
+        w0 = word_at<true>(a, nullptr);
+        w1 = word_at<true>(a + 4, nullptr);
+      }
+    } else {
+      ok = b != nullptr;
+      if (ok) {
+        const unsigned short* sa = reinterpret_cast<const unsigned short*>(b + kd.off2) + prow * kd.ng + sg0;
+        s0 = sa[0];
+        s1 = split < 8 ? sa[1] : s0;
+        if (b4) {
+          w0 = word_at<false>(0, b + kd.off0 + prow * kd.pitch + (k0 >> 1));
+        } else {
+          const uint8_t* a = b + kd.off1 + prow * kd.nb4 + 3 * (j0 >> 3);
+          w0 = word_at<false>(0, a);
+          w1 = word_at<false>(0, a + 4);
+        }
+      }
+    }
+    if (!ok) { s0 = 0; s1 = 0; }
+    uint4 z;
+    if (b4) {
+      // nibbles of the 4 bytes at k0/2: (n xor 8) = code + 8 under 0x64 -> 1032 + code
+      const uint32_t raw = w0, hi = raw >> 4;
+      const __half2 off = __half2half2(__ushort_as_half(0x6408));
+      const __half2 s2 = __half2half2(__ushort_as_half(s0));
+      z.x = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0400) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+      z.y = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0501) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+      z.z = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0602) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+      z.w = h2_bits(__hmul2(__hsub2(bits_h2((__byte_perm(raw, hi, 0x0703) & 0x000F000Fu) ^ 0x64086408u), off), s2));
+    } else {
+      // the group's 24 bits: codes j0 .. j0+7 start at bit 3 (j0 mod 8) of the word pair
+      const uint64_t win = (static_cast<uint64_t>(w1) << 32) | w0;
+      const uint32_t c24 = static_cast<uint32_t>(win >> (3 * (j0 & 7)));
+      const __half2 off = __half2half2(__ushort_as_half(0x6404));  // 1028
+      uint32_t zz[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = (c24 >> (6 * q)) & 7u, hi = (c24 >> (6 * q + 3)) & 7u;
+        const __half2 s2 = __halves2half2(__ushort_as_half(2 * q < split ? s0 : s1),
+                                          __ushort_as_half(2 * q + 1 < split ? s0 : s1));
+        zz[q] = h2_bits(__hmul2(__hsub2(bits_h2((lo | (hi << 16)) ^ 0x64046404u), off), s2));
+      }
+      z = make_uint4(zz[0], zz[1], zz[2], zz[3]);
+    }
+    st_shared_v4(dst + sw128_offset(r, ch), z);
+  }
+  return true;
+}
+
+template <bool SMEM, bool H43, class BaseFn>
 __device__ __forceinline__ void dequant_rows8(uint32_t dst, const LatDesc& kd, int k0, int ch,
                                               int row0, BaseFn key_base, uint32_t safe = 0) {
-  const bool i8 = k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0;
-  const bool i4 = !i8 && k0 >= kd.n8 && ((k0 - kd.n8) & 7) == 0 && k0 + 8 <= kd.rank &&
+  if constexpr (H43) {
+    if (dequant_rows8_h43<SMEM>(dst, kd, k0, ch, row0, key_base, safe)) return;
+  }
+  const bool i8 = !H43 && k0 + 8 <= kd.n8 && (kd.n8 & 7) == 0;
+  const bool i4 = !H43 && !i8 && k0 >= kd.n8 && ((k0 - kd.n8) & 7) == 0 && k0 + 8 <= kd.rank &&
                   (kd.nb4 & 3) == 0;
   if (i8 || i4) {
     const int j0 = k0 - kd.n8;
@@ -305,9 +443,9 @@ __device__ __forceinline__ void dequant_rows8(uint32_t dst, const LatDesc& kd, i
       const auto b = key_base(it, r);
       uint4 z = make_uint4(0, 0, 0, 0);
       if constexpr (SMEM) {
-        if (b != kNoRow) z = dequant8_at(smem_generic(b), kd, r & 63, k0);
+        if (b != kNoRow) z = dequant8_at<H43>(smem_generic(b), kd, r & 63, k0);
       } else {
-        if (b) z = dequant8_at(b, kd, r & 63, k0);
+        if (b) z = dequant8_at<H43>(b, kd, r & 63, k0);
       }
       st_shared_v4(dst + sw128_offset(r, ch), z);
     }
@@ -966,7 +1104,7 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
           const uint32_t codes = smem_u32(sCodes) + static_cast<uint32_t>(cb * 2 * kreg);
           const uint32_t pb0 = U.page0 >= 0 ? codes : kNoRow;
           const uint32_t pb1 = U.page1 >= 0 ? codes + static_cast<uint32_t>(kreg) : kNoRow;
-          dequant_rows8<true>(smem_u32(sA + kb * kAStage), kd, kb * 64 + ch * 8, ch, tid >> 3,
+          dequant_rows8<true, FMT == FMT_HAD43>(smem_u32(sA + kb * kAStage), kd, kb * 64 + ch * 8, ch, tid >> 3,
                               [&](int it, int r) -> uint32_t {
                                 return r < U.nvalid ? (it < 4 ? pb0 : pb1) : kNoRow;
                               }, codes);
@@ -1015,14 +1153,14 @@ __global__ void __launch_bounds__(Fmt<FMT>::kWarps * 32, 1)
               const uint32_t codes = smem_u32(sCodes);
               const uint32_t pb0 = U.page0 >= 0 ? codes : kNoRow;
               const uint32_t pb1 = U.page1 >= 0 ? codes + static_cast<uint32_t>(kreg) : kNoRow;
-              dequant_rows8<true>(dst, kd, kb * 64 + ch * 8, ch, tid >> 3,
+              dequant_rows8<true, FMT == FMT_HAD43>(dst, kd, kb * 64 + ch * 8, ch, tid >> 3,
                                   [&](int it, int r) -> uint32_t {
                                     return r < U.nvalid ? (it < 4 ? pb0 : pb1) : kNoRow;
                                   }, codes);
             } else {
               const uint8_t* gb0 = U.page0 >= 0 ? p.cache + (long long)U.page0 * p.page_bytes : nullptr;
               const uint8_t* gb1 = U.page1 >= 0 ? p.cache + (long long)U.page1 * p.page_bytes : nullptr;
-              dequant_rows8<false>(dst, p.key, kb * 64 + ch * 8, ch, tid >> 3,
+              dequant_rows8<false, FMT == FMT_HAD43>(dst, p.key, kb * 64 + ch * 8, ch, tid >> 3,
                                    [&](int it, int r) -> const uint8_t* {
                                      return r < U.nvalid ? (it < 4 ? gb0 : gb1) : nullptr;
                                    });
@@ -1222,7 +1360,7 @@ static cudaError_t launch_hd(int hd, int G, const DecodeParams& p, const CUtenso
 cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
                           const CUtensorMap& tmA, const CUtensorMap& tmB, int grid,
                           cudaStream_t s) {
-  const int res = fmt == STARKV_FMT_MIXED ? p.a_resident : 0;
+  const int res = (fmt == STARKV_FMT_MIXED || fmt == STARKV_FMT_HAD43) ? p.a_resident : 0;
   if (p.cta_group == 2) {
     switch (fmt) {
       case STARKV_FMT_BF16: return launch_hd<FMT_BF16, 2>(head_dim, G, p, tmA, tmB, grid, s);
@@ -1230,6 +1368,10 @@ cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
         return res == 1   ? launch_hd<FMT_MIXED, 2, 1>(head_dim, G, p, tmA, tmB, grid, s)
                : res == 2 ? launch_hd<FMT_MIXED, 2, 2>(head_dim, G, p, tmA, tmB, grid, s)
                           : launch_hd<FMT_MIXED, 2, 0>(head_dim, G, p, tmA, tmB, grid, s);
+      case STARKV_FMT_HAD43:
+        return res == 1   ? launch_hd<FMT_HAD43, 2, 1>(head_dim, G, p, tmA, tmB, grid, s)
+               : res == 2 ? launch_hd<FMT_HAD43, 2, 2>(head_dim, G, p, tmA, tmB, grid, s)
+                          : launch_hd<FMT_HAD43, 2, 0>(head_dim, G, p, tmA, tmB, grid, s);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -1240,6 +1382,10 @@ cudaError_t launch_decode(int fmt, int head_dim, int G, const DecodeParams& p,
       return res == 1   ? launch_hd<FMT_MIXED, 1, 1>(head_dim, G, p, tmA, tmB, grid, s)
              : res == 2 ? launch_hd<FMT_MIXED, 1, 2>(head_dim, G, p, tmA, tmB, grid, s)
                         : launch_hd<FMT_MIXED, 1, 0>(head_dim, G, p, tmA, tmB, grid, s);
+    case STARKV_FMT_HAD43:
+      return res == 1   ? launch_hd<FMT_HAD43, 1, 1>(head_dim, G, p, tmA, tmB, grid, s)
+             : res == 2 ? launch_hd<FMT_HAD43, 1, 2>(head_dim, G, p, tmA, tmB, grid, s)
+                        : launch_hd<FMT_HAD43, 1, 0>(head_dim, G, p, tmA, tmB, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -130,10 +130,6 @@ extern "C" starkv_status starkv_decode_attention_noalloc(
   starkv_sizes sz;
   starkv_status st = starkv_alloc(lay, 0, batch < 0 ? 0 : batch, max_pages, 0, &sz);
   if (st != STARKV_OK) return st;
-  if (lay->cfg.fmt == STARKV_FMT_HAD43) {  // refused before the scratch lookup touches a device
-    starkv::set_error_message("decode of the had43 format is not implemented yet");
-    return STARKV_ERR_UNSUPPORTED;
-  }
   if (sz.decode_workspace_bytes > kScratchBytes) {
     starkv::set_error_message(
         "starkv_decode_attention_noalloc: the partial records of this call need " +

@@ -159,34 +159,20 @@ def test_store_rejects_token_counts_past_32_bit_warp_numbering(lib):
     assert st == L.ERR_INVALID_ARG
 
 
-def test_had43_decode_is_refused_before_touching_the_device(lib):
-    # the pages' own format has its page layout (above), store and read-back, but no decode
-    # kernel yet: the decode calls refuse it before any device call (the pointers are never
-    # used)
-    lay = api.layout_init(api.make_config(32, 8, 128, 4096, 256, [32] * 8, "had43", 500000.0))
-    s = L.Sizes()
-    assert lib.starkv_alloc(ctypes.byref(lay), 4, 1, 4, 8, ctypes.byref(s)) == L.OK
-    assert s.cache_bytes == 4 * lay.page_bytes
-    fake = ctypes.c_void_p(1 << 20)
-    calls = {
-        "decode_attention": lambda: lib.starkv_decode_attention(
-            ctypes.byref(lay), fake, fake, 1, fake, 1, fake, 1, fake, fake, fake, 1 << 30, fake,
-            fake, 1 << 30, None, fake, None),
-        "decode_partials": lambda: lib.starkv_decode_partials(
-            ctypes.byref(lay), fake, fake, 1, fake, 1, fake, 1, fake, fake, 1 << 30, fake,
-            1 << 30, None, fake, None),
-        "decode_combine": lambda: lib.starkv_decode_combine(ctypes.byref(lay), fake, 1, 1, fake,
-                                                            fake, 1 << 30, fake, None),
-        "decode_attention_noalloc": lambda: lib.starkv_decode_attention_noalloc(
-            ctypes.byref(lay), fake, fake, 1, fake, 1, fake, 1, fake, fake, fake, 1 << 30, fake,
-            None, fake, None),
-        "decode_plan_query": lambda: lib.starkv_decode_plan_query(ctypes.byref(lay), 1, 1, None,
-                                                                  148, 232448,
-                                                                  ctypes.byref(L.DecodePlan())),
-    }
-    for name, call in calls.items():
-        assert call() == L.ERR_UNSUPPORTED, name
-        assert b"had43" in lib.starkv_last_error(), name
+def test_had43_decode_plans_like_int8_int4(lib):
+    """The pages' own format decodes through the int8/int4 machinery: the same key modes
+    (resident operand at rank <= 256, staged codes above), CTA pairs and chunking."""
+    for rk, rv, batch, pages, mode, cg in [(256, [32] * 8, 32, 512, 1, 2),
+                                           (1024, [32] * 32, 16, 256, 2, 1)]:
+        hkv = len(rv)
+        lay_m = api.layout_init(api.make_config(32, hkv, 128, 4096, rk, rv, "mixed", 1e4))
+        lay_h = api.layout_init(api.make_config(32, hkv, 128, 4096, rk, rv, "had43", 1e4))
+        pm = api.decode_plan(lay_m, batch, pages)
+        ph = api.decode_plan(lay_h, batch, pages)
+        assert (ph.key_mode, ph.cta_group) == (mode, cg)
+        assert (ph.chunk_cols, ph.n_chunks, ph.n_ranges, ph.grid) == \
+            (pm.chunk_cols, pm.n_chunks, pm.n_ranges, pm.grid)
+        assert 120 * 1024 <= ph.smem_bytes <= 232448
 
 
 def test_alloc_rejects_a_cache_size_past_size_t(lib):
