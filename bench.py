@@ -252,7 +252,8 @@ def time_graph(graph, flush, stream, steps, torch):
 
 def append_bench(w, lay, pk, steps, dev, torch, api, W, wl, seq, pos, x_new, flush, stream):
     """The latent write on its own: (1) the decode-step append of this workload's batch (one
-    new token per sequence: projection of B rows, then quantise/pack/scatter), bounded by
+    new token per sequence: projection of B rows, then quantise/pack/scatter; up to 32 tokens
+    in a bf16-operand format this is the one fused launch of append_gemv_kernel), bounded by
     reading A from HBM; (2) an 8192-token prefill chunk of the long-context GQA layer,
     bounded by the tensor cores.  Each as tokens/s and as a fraction of its bound."""
     out = {}
@@ -274,11 +275,15 @@ def append_bench(w, lay, pk, steps, dev, torch, api, W, wl, seq, pos, x_new, flu
         t_tc = flop / (pk["bf16_tflops"] * NOMINAL_RATIO["bf16" if es == 2 else "tf32"] * 1e12)
         t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
         bound = "tensor" if t_tc >= t_hbm else "hbm"
+        # starkv_append's dispatch: a step of at most 32 tokens with bf16 operands is the fused
+        # projection + store kernel, anything else the projection kernel then the store kernel
+        fused = lay_.cfg.fmt != api.L.FMT["f32"] and n <= 32
+        kernels = ["append_gemv_kernel"] if fused else ["project_kernel", "store_kernel"]
         out[name] = {"tokens": n, "us_median": ms * 1000.0, "tokens_per_s": n / (ms / 1000.0),
                      "bound": bound, "bound_us": max(t_tc, t_hbm) * 1e6,
                      "frac_of_bound": max(t_tc, t_hbm) / (ms / 1000.0),
-                     "flop": flop, "bytes": nbytes, "kernels": ["project_kernel", "store_kernel"]}
-        return 2 * steps
+                     "flop": flop, "bytes": nbytes, "kernels": kernels}
+        return len(kernels) * steps
 
     launches += one("decode_step", lay, x_new, wl.A_t, seq, pos, wl.block_table, wl.lc.cache,
                     wl.lc.append_ws, wl.lc.status)

@@ -428,6 +428,30 @@ starkv_status starkv_append(const starkv_layout* lay, const void* x, int32_t n_t
   if (st != STARKV_OK) return st;
   const int fmt = lay->cfg.fmt;
   const int es = elem_size(fmt);
+  // A decode step (at most 32 tokens, bf16 operands): one launch that projects on the tensor
+  // cores and stores, with the k-split partials added in a cluster's shared memory.  The
+  // k-slice is the smallest of d_model / {8, 4, 2, 1} that is a multiple of 64 columns and
+  // keeps at least 256 (d_model itself when none does).
+  if (fmt != STARKV_FMT_F32 && n_tok <= kGemvMaxTokens) {
+    const int dm = lay->cfg.d_model;
+    int ks = 8;
+    while (ks > 1 && (dm % (64 * ks) != 0 || dm / ks < 256)) ks /= 2;
+    if (append_gemv_smem(dm / ks, n_tok) <= info.smem_optin) {
+      GemvParams gp;
+      std::memset(&gp, 0, sizeof(gp));
+      gp.sp = sp;
+      gp.sp.latents_out = latents_out;
+      gp.x = reinterpret_cast<const __nv_bfloat16*>(x);
+      gp.A_t = reinterpret_cast<const __nv_bfloat16*>(A_t);
+      gp.d_model = dm;
+      gp.ks = ks;
+      gp.kslice = dm / ks;
+      gp.timeout_ns = 4000000000ull;
+      cudaError_t e = launch_append_gemv(gp, reinterpret_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return cuda_fail(e, "decode-step append launch");
+      return STARKV_OK;
+    }
+  }
   ProjParams pp;
   std::memset(&pp, 0, sizeof(pp));
   proj_plan(lay, n_tok, pp.kb_total, pp.kb_per_split, pp.nsplit);

@@ -102,6 +102,21 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 
 cudaError_t launch_store(const StoreParams& p, cudaStream_t s);
 
+// Fused latent write of a decode step (at most 32 tokens, bf16 operands): projection on the
+// tensor cores and the store in one launch, one cluster of ks CTAs (k-slices) per 32-channel
+// chunk.
+struct GemvParams {
+  StoreParams sp;              // the store (latents, chunks, tokens, pages, status)
+  const __nv_bfloat16* x;      // [n_tok][d_model]
+  const __nv_bfloat16* A_t;    // [proj_cols][d_model]
+  int d_model, kslice, ks;     // d_model = ks * kslice, kslice a multiple of 16
+  int row_bytes;               // set by the launcher
+  unsigned long long timeout_ns;
+};
+constexpr int kGemvMaxTokens = 32;
+size_t append_gemv_smem(int kslice, int n_tok);
+cudaError_t launch_append_gemv(const GemvParams& p, cudaStream_t s);
+
 // Weight absorption (attention output projection folded into the value up-projection).
 struct AbsorbParams {
   const float* Bv;  // [R_v][d]

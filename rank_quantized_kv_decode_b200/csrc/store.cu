@@ -13,51 +13,13 @@
 // the leading ceil(r/5) channels are 4-bit codes (qmax 7, two per byte as above), the rest
 // 3-bit codes (qmax 3), eight per 3 bytes as the little-endian 24-bit word
 // sum_i (code_i & 7) 8^i; same scale rule, groups of 32 restarting at the 3-bit block.
-#include "internal.cuh"
+#include "store_dev.cuh"
 
 namespace starkv {
 
 namespace {
 
-__device__ __forceinline__ float warp_max_abs(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-// fp16 scale of a group (saturating) and the code of value c.
-__device__ __forceinline__ __half group_scale(float amax, float qmax) {
-  __half h = __float2half_rn(__fdiv_rn(amax, qmax));
-  if (__hisinf(h)) h = __ushort_as_half(static_cast<unsigned short>(0x7BFF));
-  return h;
-}
-__device__ __forceinline__ int quant_code(float c, float s, int qmax) {
-  if (s == 0.f) return 0;
-  const int q = __float2int_rn(__fdiv_rn(c, s));
-  return max(-qmax, min(qmax, q));
-}
-
-struct TokenSlot {
-  uint8_t* page;  // nullptr if the token's page or position is invalid
-  int slot;
-};
-
-__device__ __forceinline__ TokenSlot locate(const StoreParams& p, int n, int li, int lane) {
-  const int b = p.tok_seq[n], pos = p.tok_pos[n];
-  TokenSlot t{nullptr, 0};
-  if (b < 0 || b >= p.batch || pos < 0 || pos >= p.max_pages * kPage) {
-    if (lane == 0 && li == 0 && p.status) atomicOr(p.status, STARKV_DEV_BOUNDS);
-    return t;
-  }
-  const int pg = p.block_table[(long long)b * p.max_pages + pos / kPage];
-  if (pg < 0 || pg >= p.num_pages) {
-    if (lane == 0 && li == 0 && p.status) atomicOr(p.status, STARKV_DEV_BOUNDS);
-    return t;
-  }
-  t.page = p.cache + (long long)pg * p.page_bytes;
-  t.slot = pos % kPage;
-  return t;
-}
+using namespace store_dev;
 
 // Sum of the split-K partials of one value, in split order (deterministic).  Up to 16 loads
 // are issued before the first add, so a decode step's partials arrive in one round trip.
@@ -83,88 +45,10 @@ __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ Stor
   const int lane = threadIdx.x & 31;
   if (gw >= p.n_tok * p.chunks_per_token) return;  // whole warp
   const int n = gw / p.chunks_per_token;
-  const int ck = gw % p.chunks_per_token;
-  int li = 0;
-  while (p.chunk_start[li + 1] <= ck) ++li;
-  const int cl = ck - p.chunk_start[li];  // chunk within the latent
-  const LatDesc& d = p.lat[li];
-  const float* src = p.src + (long long)n * p.proj_cols + d.col;
-  float* lout = p.latents_out ? p.latents_out + (long long)n * p.proj_cols + d.col : nullptr;
-  // this lane's channel of the chunk; the partial sums are loaded before the page lookup so
-  // that both round trips overlap
-  const bool plain = p.fmt == STARKV_FMT_F32 || p.fmt == STARKV_FMT_BF16;
-  const bool is8 = !plain && cl < d.g8;
-  const int n4 = d.rank - d.n8;
-  const int j = (plain || is8) ? 0 : (cl - d.g8) * 32 + lane;  // int4 channel index
-  const int i = (plain || is8) ? cl * 32 + lane : d.n8 + j;    // channel in the latent
-  const bool in = plain ? i < d.rank : (is8 ? i < d.n8 : j < n4);
-  const float c = in ? split_sum(src + i, p.split_stride, p.nsplit) : 0.f;
-  if (lout && in) lout[i] = c;
-  const TokenSlot ts = locate(p, n, (li == 0 && cl == 0) ? 0 : 1, lane);
-
-  if (plain) {
-    if (!in || !ts.page) return;
-    uint8_t* dst = ts.page + d.off0 + ts.slot * d.pitch;
-    if (p.fmt == STARKV_FMT_F32)
-      reinterpret_cast<float*>(dst)[i] = c;
-    else
-      reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(c);
-    return;
-  }
-  __half* sc = ts.page ? reinterpret_cast<__half*>(ts.page + d.off2) + ts.slot * d.ng : nullptr;
-  if (p.fmt == STARKV_FMT_HAD43) {
-    const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
-    if (is8) {
-      // 4-bit group cl: channels [32 cl, min(32 cl + 32, n8)), d.pitch packed bytes per token
-      const __half h = group_scale(amax, 7.f);
-      const int nib = quant_code(c, __half2float(h), 7) & 15;
-      const int hi = __shfl_down_sync(0xffffffffu, nib, 1);
-      if (ts.page && in && (i & 1) == 0) {
-        const int byte = nib | ((i + 1 < d.n8 ? hi : 0) << 4);
-        (ts.page + d.off0)[ts.slot * d.pitch + (i >> 1)] = static_cast<uint8_t>(byte);
-      }
-      if (ts.page && lane == 0) sc[cl] = h;
-    } else {
-      // 3-bit group gi: channels n8 + [32 gi, min(32 gi + 32, n4)); lanes 8k..8k+7 form word
-      // k of the group (lanes past n4 hold c = 0, code 0: the padding of the last word)
-      const int gi = cl - d.g8;
-      const __half h = group_scale(amax, 3.f);
-      const int code = quant_code(c, __half2float(h), 3) & 7;
-      uint32_t w = static_cast<uint32_t>(code) << (3 * (lane & 7));
-      w |= __shfl_xor_sync(0xffffffffu, w, 1);
-      w |= __shfl_xor_sync(0xffffffffu, w, 2);
-      w |= __shfl_xor_sync(0xffffffffu, w, 4);
-      if (ts.page && in && (lane & 7) == 0) {
-        uint8_t* dst = ts.page + d.off1 + ts.slot * d.nb4 + 3 * (j >> 3);
-        dst[0] = static_cast<uint8_t>(w);
-        dst[1] = static_cast<uint8_t>(w >> 8);
-        dst[2] = static_cast<uint8_t>(w >> 16);
-      }
-      if (ts.page && lane == 0) sc[d.g8 + gi] = h;
-    }
-    return;
-  }
-  if (is8) {
-    // int8 group cl: channels [32 cl, min(32 cl + 32, n8))
-    const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
-    const __half h = group_scale(amax, 127.f);
-    const int q = quant_code(c, __half2float(h), 127);
-    if (ts.page && in) reinterpret_cast<int8_t*>(ts.page + d.off0)[ts.slot * d.n8 + i] = static_cast<int8_t>(q);
-    if (ts.page && lane == 0) sc[cl] = h;
-  } else {
-    // int4 group gi: channels n8 + [32 gi, min(32 gi + 32, n4))
-    const int gi = cl - d.g8;
-    const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
-    const __half h = group_scale(amax, 7.f);
-    const int q = quant_code(c, __half2float(h), 7);
-    const int nib = q & 15;
-    const int hi = __shfl_down_sync(0xffffffffu, nib, 1);
-    if (ts.page && in && (j & 1) == 0) {
-      const int byte = nib | ((j + 1 < n4 ? hi : 0) << 4);
-      (ts.page + d.off1)[ts.slot * d.nb4 + (j >> 1)] = static_cast<uint8_t>(byte);
-    }
-    if (ts.page && lane == 0) sc[d.g8 + gi] = h;
-  }
+  const ChunkLane q = chunk_lane(p, gw % p.chunks_per_token, lane);
+  const float* src = p.src + (long long)n * p.proj_cols + p.lat[q.li].col;
+  const float c = q.in ? split_sum(src + q.i, p.split_stride, p.nsplit) : 0.f;
+  store_value(p, q, n, lane, c);
 }
 
 // One warp per (token, latent): stored value -> fp32 (scale * code for the mixed format).

@@ -49,26 +49,33 @@ def test_append_projection_and_store(index, n_tok):
     proj_tol = 1e-4
     proj_err = np.abs(got - want)
     assert np.max(proj_err / scale) < proj_tol
-    # stored values: read back and compare with the oracle's storage of its own latents
+    # stored values, read back: (1) bit-exact against the oracle's storage of the GPU's own
+    # fp32 latents (the quantiser and the packing are exact functions of their input)
     back = torch.empty_like(lat_out)
     api.dequant(lay, lc.cache, seq, pos, table, back, lc.status)
     torch.cuda.synchronize()
+    assert lc.status.item() == 0
     stored_gpu = back.cpu().numpy().astype(np.float64)
+    Ck_g, Cv_g = ref.stored(lat_out.cpu().numpy())
+    np.testing.assert_array_equal(stored_gpu, np.concatenate([Ck_g] + Cv_g, axis=1))
+    # (2) against the oracle's storage of its own fp64 latents: the projections differ by the
+    # fp32 rounding above, and the quantiser is discontinuous (a group's absmax near an fp16
+    # rounding boundary of its scale moves the whole group to the neighbouring scale), so each
+    # stored value may differ by at most one quantisation step of either scale (mixed), or by
+    # the projection error plus one bf16 spacing (bf16), or the projection error (f32)
     Ck, Cv = ref.stored(want.astype(np.float32))
     stored_ref = np.concatenate([Ck] + Cv, axis=1)
     diff = np.abs(stored_gpu - stored_ref)
     if fmt == "mixed":
-        # one quantisation step at most, and rarely
         cols = np.concatenate([[0], np.cumsum([st.key_rank] + st.value_ranks)])
-        frac = np.mean(diff > 0)
-        assert frac < 2e-3, f"{frac:.2e} of stored values differ"
         for li in range(len(cols) - 1):
-            part = want[:, cols[li]:cols[li + 1]].astype(np.float32)
-            _, _, sc = O.quantize_rows(part, part.shape[1])
-            step = sc.astype(np.float64).max(axis=1, keepdims=True)
-            assert np.all(diff[:, cols[li]:cols[li + 1]] <= 1.01 * step + 1e-12)
+            sl = slice(cols[li], cols[li + 1])
+            _, _, sc_ref = O.quantize_rows(want[:, sl].astype(np.float32), cols[li + 1] - cols[li])
+            _, _, sc_gpu = O.quantize_rows(got[:, sl].astype(np.float32), cols[li + 1] - cols[li])
+            step = np.maximum(sc_ref.astype(np.float64), sc_gpu.astype(np.float64)).max(axis=1, keepdims=True)
+            assert np.all(diff[:, sl] <= 1.01 * step + 1e-12)
+        print(f"values differing from the storage of the fp64 latents: {np.mean(diff > 0):.2e}")
     else:
-        # the store itself is exact (f32) or one rounding (bf16): the difference is the
-        # projection error plus at most one storage ulp
-        ulp = np.abs(stored_ref) * (2.0 ** -8 if fmt == "bf16" else 2.0 ** -23)
-        assert np.all(diff <= proj_err * (1 + 1e-6) + ulp)
+        mag = np.maximum(np.abs(stored_ref), np.abs(stored_gpu))
+        spacing = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - (7 if fmt == "bf16" else 23))
+        assert np.all(diff <= proj_err * (1 + 1e-6) + spacing)
