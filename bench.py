@@ -311,6 +311,40 @@ def append_bench(w, lay, pk, steps, dev, torch, api, W, wl, seq, pos, x_new, flu
     return out, launches
 
 
+def hybrid_bench(pk, steps, torch, W, flush, stream):
+    """Decode with the pages' own assignment (keys head-wise, values joint) on a cache of the
+    largest workload's size: 32 sequences x 32768 tokens, GQA 32/8, d 128, int8/int4, per-head
+    key ranks 16-48 (total 256) and a joint value rank of 256.  Split + combine timed per step
+    (CUDA events, L2 flushed between steps), as KV tokens/s and against its bound."""
+    hw = W.build_hybrid()
+    for _ in range(3):
+        W.decode_hybrid(hw)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        W.decode_hybrid(hw)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert hw.lc.status.item() == 0
+    ms = float(np.median([a.elapsed_time(b) for a, b in evs]))
+    w, lay = hw.w, hw.lay
+    tok = w["batch"] * w["context"]
+    H, d, rv = w["n_q_heads"], w["head_dim"], w["value_rank"]
+    # per token: K_g = C_k,g B_k,g for every KV head, the scores, and P C_v in the joint space
+    flop = tok * (2.0 * sum(w["key_ranks"]) * d + 2.0 * H * d + 2.0 * H * rv)
+    nbytes = float(tok * lay.token_bytes)
+    t_tc = flop / (pk["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    return {"workload": w["name"], "us_median": ms * 1000.0, "kv_tokens_per_s": tok / (ms / 1000.0),
+            "bytes": nbytes, "flop": flop, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "bound_us": max(t_tc, t_hbm) * 1e6, "achieved_gbs": nbytes / (ms / 1000.0) / 1e9,
+            "frac_of_hbm": t_hbm / (ms / 1000.0), "frac_of_bound": max(t_tc, t_hbm) / (ms / 1000.0),
+            "kernels": ["hybrid_split_kernel", "hybrid_combine_kernel"]}, 2 * steps
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -320,6 +354,7 @@ def main():
     ap.add_argument("--workload", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-append-bench", action="store_true")
+    ap.add_argument("--no-hybrid-bench", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -479,6 +514,12 @@ def main():
                                   flush, stream)
         app["clocks"] = aclk.summary()
         line["append"] = app
+        gpu_launches += n
+    if not args.no_hybrid_bench and world == 1:
+        with ClockSampler(local) as hclk:
+            hyb, n = hybrid_bench(pk, args.steps, torch, W, flush, stream)
+        hyb["clocks"] = hclk.summary()
+        line["hybrid"] = hyb
         gpu_launches += n
     line["gpu_launches"] = gpu_launches
     line["gpu_launches_e2e"] = e2e_launches

@@ -20,6 +20,9 @@
  *       a_h = p C_v,g(h), o_h = a_h B_v,g(h).
  *   Optionally with the value up-projection folded into the output projection
  *   (Methodology §2): y = sum_h a_h (B_v,g(h) W_o,h).
+ *   And with the pages' own assignment (Methodology §2, "Hybrid Decomposition Strategy"):
+ *   keys head-wise (c_k,g = x A_k,g per KV head), values joint (one c_v = x A_v), decoded by
+ *   starkv_hybrid_decode.
  *
  * Conventions shared by every entry point:
  *   - The caller owns all memory.  The library never allocates device memory, never
@@ -95,8 +98,31 @@ typedef struct {
   double rope_theta;   /* RoPE base                                                     */
 } starkv_config;
 
-/* One latent's place in a page.  Latent 0 is the key latent, latent 1+g the value latent
- * of KV head g.  Each block is token-major ([token][...]) and starts on a 16-byte
+/* Which latents a layout holds (starkv_layout.assignment). */
+#define STARKV_ASSIGN_JOINT_KEYS 0 /* starkv_layout_init: latent 0 the joint key latent, latent
+                                      1+g the value latent of KV head g                    */
+#define STARKV_ASSIGN_HYBRID 1     /* starkv_hybrid_layout_init: latent g the key latent of KV
+                                      head g, latent n_kv_heads the joint value latent     */
+
+/* The pages' own assignment (STAR-KV technical summary, Methodology §2, "Hybrid
+ * Decomposition Strategy"): keys decomposed head-wise (KV head g has its own latent of rank
+ * r_k,g and factor B_k,g, r_k,g x d), values jointly (one latent of rank r_v for all KV heads
+ * and one factor B_v, r_v x (n_kv_heads d)).  Host struct, POD. */
+typedef struct {
+  int32_t n_q_heads;  /* H; a multiple of n_kv_heads, at most 8 per KV head               */
+  int32_t n_kv_heads; /* H_kv, 1..STARKV_MAX_KV_HEADS                                       */
+  int32_t head_dim;   /* d: 64 or 128                                                      */
+  int32_t d_model;    /* hidden size of x (append); a multiple of 64                        */
+  int32_t key_rank[STARKV_MAX_KV_HEADS]; /* r_k,g: a multiple of 16 in [16, head_dim]       */
+  int32_t value_rank; /* r_v: a multiple of 16 in [16, min(2048, n_kv_heads head_dim)]      */
+  int32_t fmt;        /* starkv_fmt (every format has a layout; decode takes mixed)         */
+  int32_t page_tokens; /* must be 64                                                        */
+  double rope_theta;   /* RoPE base                                                         */
+} starkv_hybrid_config;
+
+/* One latent's place in a page.  In a joint-key layout latent 0 is the key latent, latent
+ * 1+g the value latent of KV head g; in a hybrid layout latent g is the key latent of KV
+ * head g and latent n_kv_heads the joint value latent.  Each block is token-major ([token][...]) and starts on a 16-byte
  * boundary; absent blocks have offset -1.  The quantised formats have two channel blocks,
  * the leading (more precise) one and the rest; in had43 the fields named for int8/int4 hold
  * them as follows:
@@ -110,7 +136,8 @@ typedef struct {
 typedef struct {
   int32_t rank;  /* channels r                                                          */
   int32_t col;   /* first column of this latent in the concatenated projection
-                    [c_k | c_v,0 | c_v,1 | ...] (and row in the stacked B_v for values)  */
+                    [c_k | c_v,0 | c_v,1 | ...] (and row in the stacked B_v for values);
+                    hybrid: [c_k,0 | ... | c_k,H_kv-1 | c_v]                             */
   int32_t n8;    /* mixed: int8 channels [0, n8), n8 = ceil(r/4)                         */
   int32_t n4;    /* mixed: int4 channels [n8, r)                                         */
   int32_t g8;    /* mixed: scale groups of the int8 part, ceil(n8/32)                    */
@@ -125,14 +152,18 @@ typedef struct {
 } starkv_segment;
 
 typedef struct {
-  starkv_config cfg;
+  starkv_config cfg;        /* hybrid: the shared fields of the hybrid config; key_rank and
+                               value_rank[] are 0                                      */
   int32_t n_latents;        /* 1 + n_kv_heads                                          */
-  int32_t proj_cols;        /* key_rank + value_rank_total                             */
-  int32_t value_rank_total; /* R_v = sum of value_rank                                 */
+  int32_t proj_cols;        /* key_rank + value_rank_total (hybrid: sum r_k,g + r_v)    */
+  int32_t value_rank_total; /* R_v = sum of value_rank (hybrid: r_v)                   */
   int32_t value_rank_max;
   int64_t page_bytes;       /* bytes of one page (a multiple of 16)                     */
   int64_t token_bytes;      /* stored bytes per token over all latents, no padding      */
   starkv_segment seg[1 + STARKV_MAX_KV_HEADS];
+  int32_t assignment;       /* STARKV_ASSIGN_JOINT_KEYS or STARKV_ASSIGN_HYBRID          */
+  int32_t reserved;         /* 0                                                        */
+  starkv_hybrid_config hybrid; /* the config of a hybrid layout; all zero otherwise     */
 } starkv_layout;
 
 /* Buffer sizes for starkv_alloc. */
@@ -158,6 +189,16 @@ typedef struct {
 /* Fill ``out`` from ``cfg``: per-latent mixed split, block offsets, page size.
  * Host only, pure.  INVALID_ARG / UNSUPPORTED for configurations outside the limits above. */
 STARKV_API starkv_status starkv_layout_init(const starkv_config* cfg, starkv_layout* out);
+
+/* The layout of the hybrid assignment (keys head-wise, values joint; STAR-KV technical
+ * summary, Methodology §2).  Latents in page order: the key latents of KV heads 0..H_kv-1,
+ * then the joint value latent; each placed exactly as starkv_layout_init places a latent of
+ * the same rank and format.  Host only, pure; INVALID_ARG / UNSUPPORTED outside the limits
+ * of starkv_hybrid_config.  starkv_alloc, starkv_rope_init, starkv_quant_pack, starkv_append
+ * and starkv_dequant take the result (the latents are generic there); the joint-key decode
+ * calls refuse it with UNSUPPORTED, starkv_hybrid_decode takes only it. */
+STARKV_API starkv_status starkv_hybrid_layout_init(const starkv_hybrid_config* cfg,
+                                                   starkv_layout* out);
 
 /* Sizes of the caller-allocated buffers (nothing is allocated).  ``max_pages`` is the
  * row length of the block table; positions run below max_pages * page_tokens.
@@ -342,6 +383,37 @@ STARKV_API starkv_status starkv_decode_attention_noalloc(
     const int32_t* block_table, int32_t max_pages, const int32_t* seq_lens, int32_t batch,
     const void* Bk_t, const float* Bv, const void* rope_table, size_t rope_table_bytes, float* out,
     const starkv_decode_opts* opts, int32_t* dev_status, starkv_stream_t stream);
+
+/* Single-token decode attention with the hybrid assignment (STAR-KV technical summary,
+ * Methodology §2: keys head-wise, values joint).  For query head h of KV head g = h / G:
+ *   K_g = C_k,g B_k,g, RoPE on K_g and on q_h (position seq_len-1), p = softmax(q' K'^T / sqrt(d)),
+ *   a_h = p C_v (the joint value latent space, r_v wide), o_h = a_h B_v[:, g d : (g+1) d].
+ *   lay        a layout from starkv_hybrid_layout_init, fmt mixed (int8/int4); other formats
+ *              UNSUPPORTED
+ *   q          device bf16 [batch][H][d], before RoPE
+ *   Bk_t       device fp16: for each KV head g in order, the block [d][r_k,g] whose row n is
+ *              column n of B_k,g; block g starts at element d * (r_k,0 + ... + r_k,g-1)
+ *   Bv         device fp32 [r_v][H_kv d] (B_v itself)
+ *   rope_table device, from starkv_rope_init with max_pages >= this call's max_pages
+ *   out        device fp32 [batch][H][d]; a sequence of length 0 gives zeros
+ *   workspace  device, >= decode_workspace_bytes of starkv_alloc for this batch/max_pages
+ *              (per (sequence, page range, query head): m, l and the r_v-wide a)
+ * Two launches: a split kernel (one CTA per SM, looping over (sequence, page range) units;
+ * per 64-token page: a bulk copy of the page, int8/int4 codes to fp16, K_g on the tensor
+ * cores (mma.sync, fp32 accumulation), RoPE, scores on the tensor cores from the rotated keys
+ * split into two fp16 parts, online softmax, P C_v on the tensor cores) and a combine
+ * (log-sum-exp merge of the page ranges, then o_h = a_h B_v,g).  Limits of the kernel
+ * (UNSUPPORTED, nothing launched): n_kv_heads <= 16, H <= 64, ceil(H/16) ceil(r_v/64) <= 8,
+ * a page below 1 MiB, and the shared-memory plan (all B_k,g resident) within the device's
+ * per-block limit.  Errors in *dev_status as for starkv_decode_attention. */
+STARKV_API starkv_status starkv_hybrid_decode(const starkv_layout* lay, const void* q,
+                                              const void* cache, int64_t num_pages,
+                                              const int32_t* block_table, int32_t max_pages,
+                                              const int32_t* seq_lens, int32_t batch,
+                                              const void* Bk_t, const float* Bv,
+                                              const void* rope_table, size_t rope_table_bytes,
+                                              float* out, void* workspace, size_t workspace_bytes,
+                                              int32_t* dev_status, starkv_stream_t stream);
 
 /* Failure-detection check of the in-kernel bounded waits: one CTA holds TMEM and waits on a
  * barrier that nothing completes.  After ``timeout_ms`` (1..10000) the wait gives up, the CTA

@@ -210,6 +210,14 @@ def page_layout(fmt: str, key_rank: int, value_ranks, page_tokens: int = 64) -> 
                 value_ranks=[int(r) for r in value_ranks])
 
 
+def hybrid_page_layout(fmt: str, key_ranks, value_rank: int, page_tokens: int = 64) -> dict:
+    """Byte layout of a page with the hybrid assignment (STAR-KV technical summary,
+    Methodology §2: keys head-wise, values joint): the key latents of KV heads 0..H_kv-1, then
+    the joint value latent, each placed exactly as page_layout places a latent of its rank."""
+    ranks = [int(r) for r in key_ranks] + [int(value_rank)]
+    return page_layout(fmt, ranks[0], ranks[1:], page_tokens)
+
+
 def mixed_bits_per_channel(r: int) -> float:
     """Average stored bits per latent channel of the int8/int4 + fp16-scale format."""
     sp = mixed_split(r)

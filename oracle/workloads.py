@@ -148,3 +148,40 @@ def _base(index: int, need_down: bool) -> Ref:
 
 def ref_for(index: int, need_down: bool = False, **overrides) -> Ref:
     return _base(index, need_down).reshaped(**overrides)
+
+
+class HybridRef:
+    """Oracle side of the hybrid workload (keys head-wise, values joint; STAR-KV technical
+    summary, Methodology §2): the same seeded factors and latents as the device builder, the
+    oracle's own storage step, and decode_attention_hybrid."""
+
+    def __init__(self, **overrides):
+        self.w = synth.hybrid_workload(**overrides)
+        Bk, Bv = synth.hybrid_factors(self.w)
+        # the factor values the tensor cores see: B_k,g as fp16; B_v as fp32
+        self.Bk_s = [stored_factor(b, O.MIXED) for b in Bk]
+        self.Bv_s = np.asarray(Bv, np.float32).astype(np.float64)
+
+    def queries(self):
+        w = self.w
+        q = synth.gaussian(synth.rng(w["index"], "q"), (w["batch"], w["n_q_heads"], w["head_dim"]),
+                           np.float32)
+        return synth.bf16_round(q)
+
+    def stored(self, lat):
+        """Stored values (fp64) of fp32 latents [C_k,0 | ... | C_v]: ([C_k,g], C_v)."""
+        ranks = list(self.w["key_ranks"]) + [self.w["value_rank"]]
+        cols = np.concatenate([[0], np.cumsum(ranks)])
+        out = [O.stored_rows(lat[:, cols[i]:cols[i + 1]], int(ranks[i]), self.w["fmt"])
+               for i in range(len(ranks))]
+        return out[:-1], out[-1]
+
+    def expected(self, b, seq_len, heads=None, q=None):
+        if seq_len == 0:
+            n = self.w["n_q_heads"] if heads is None else len(heads)
+            return np.zeros((n, self.w["head_dim"]))
+        lat = synth.hybrid_latents(self.w, b, 0, seq_len)
+        Ck, Cv = self.stored(lat)
+        qq = (self.queries() if q is None else q)[b]
+        return O.decode_attention_hybrid(qq, Ck, Cv, self.Bk_s, self.Bv_s, self.w["rope_theta"],
+                                         self.w["n_kv_heads"], heads)

@@ -13,6 +13,7 @@ GROUP = 32
 TILE_TOKENS = 128
 
 FMT = {"f32": 0, "bf16": 1, "mixed": 2, "had43": 3}
+ASSIGN_JOINT_KEYS, ASSIGN_HYBRID = 0, 1
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BOUNDS, DEV_TIMEOUT = 1, 2
@@ -27,6 +28,12 @@ class Config(ctypes.Structure):
                 ("page_tokens", i32), ("rope_theta", f64)]
 
 
+class HybridConfig(ctypes.Structure):
+    _fields_ = [("n_q_heads", i32), ("n_kv_heads", i32), ("head_dim", i32), ("d_model", i32),
+                ("key_rank", i32 * MAX_KV_HEADS), ("value_rank", i32), ("fmt", i32),
+                ("page_tokens", i32), ("rope_theta", f64)]
+
+
 class Segment(ctypes.Structure):
     _fields_ = [("rank", i32), ("col", i32), ("n8", i32), ("n4", i32), ("g8", i32), ("g4", i32),
                 ("nb4", i32), ("pitch", i32), ("off_plain", i64), ("off_i8", i64),
@@ -36,7 +43,8 @@ class Segment(ctypes.Structure):
 class Layout(ctypes.Structure):
     _fields_ = [("cfg", Config), ("n_latents", i32), ("proj_cols", i32),
                 ("value_rank_total", i32), ("value_rank_max", i32), ("page_bytes", i64),
-                ("token_bytes", i64), ("seg", Segment * (1 + MAX_KV_HEADS))]
+                ("token_bytes", i64), ("seg", Segment * (1 + MAX_KV_HEADS)),
+                ("assignment", i32), ("reserved", i32), ("hybrid", HybridConfig)]
 
 
 class Sizes(ctypes.Structure):
@@ -56,6 +64,9 @@ class DecodePlan(ctypes.Structure):
 
 EXPORTS = {
     "starkv_layout_init": (i32, [ctypes.POINTER(Config), ctypes.POINTER(Layout)]),
+    "starkv_hybrid_layout_init": (i32, [ctypes.POINTER(HybridConfig), ctypes.POINTER(Layout)]),
+    "starkv_hybrid_decode": (i32, [ctypes.POINTER(Layout), vp, vp, i64, vp, i32, vp, i32, vp, vp,
+                                   vp, sz, vp, vp, sz, vp, vp]),
     "starkv_alloc": (i32, [ctypes.POINTER(Layout), i64, i32, i32, i32, ctypes.POINTER(Sizes)]),
     "starkv_rope_init": (i32, [ctypes.POINTER(Layout), i32, vp, sz, vp]),
     "starkv_quant_pack": (i32, [ctypes.POINTER(Layout), vp, i32, vp, vp, vp, i32, i32, vp, i64,

@@ -98,6 +98,55 @@ def layout_init(cfg: L.Config) -> L.Layout:
     return lay
 
 
+def make_hybrid_config(n_q_heads: int, n_kv_heads: int, head_dim: int, d_model: int, key_ranks,
+                       value_rank: int, fmt: str, rope_theta: float,
+                       page_tokens: int = 64) -> L.HybridConfig:
+    """Config of the hybrid assignment: one key latent per KV head (ranks ``key_ranks``), one
+    joint value latent of rank ``value_rank``."""
+    c = L.HybridConfig()
+    c.n_q_heads, c.n_kv_heads, c.head_dim, c.d_model = n_q_heads, n_kv_heads, head_dim, d_model
+    if len(key_ranks) != n_kv_heads:
+        raise ValueError("one key rank per KV head")
+    for g, r in enumerate(key_ranks):
+        c.key_rank[g] = int(r)
+    c.value_rank = int(value_rank)
+    c.fmt = L.FMT[fmt]
+    c.page_tokens = page_tokens
+    c.rope_theta = float(rope_theta)
+    return c
+
+
+def hybrid_layout_init(cfg: L.HybridConfig) -> L.Layout:
+    lay = L.Layout()
+    L.check(L.load().starkv_hybrid_layout_init(ctypes.byref(cfg), ctypes.byref(lay)),
+            "starkv_hybrid_layout_init")
+    return lay
+
+
+def hybrid_decode(lay, q, cache, block_table, seq_lens, Bk_t, Bv, rope_table, out, workspace,
+                  status, stream=None) -> None:
+    """Decode with the hybrid assignment.  Bk_t: fp16, the blocks [d][r_k,g] of the KV heads in
+    order (flat); Bv: fp32 [r_v][H_kv d]."""
+    c = lay.cfg
+    batch = seq_lens.shape[0]
+    _need(seq_lens, "seq_lens", torch.int32, ndim=1)
+    _need(block_table, "block_table", torch.int32, ndim=2)
+    if block_table.shape[0] < batch:
+        raise ValueError(f"block_table: {block_table.shape[0]} rows for {batch} sequences")
+    rk = sum(lay.seg[g].rank for g in range(c.n_kv_heads))
+    _need(q, "q", torch.bfloat16, batch * c.n_q_heads * c.head_dim)
+    _need(Bk_t, "Bk_t", torch.float16, c.head_dim * rk)
+    _need(Bv, "Bv", torch.float32, lay.value_rank_total * c.n_kv_heads * c.head_dim)
+    _need(out, "out", torch.float32, batch * c.n_q_heads * c.head_dim)
+    _need(status, "status", torch.int32, 1)
+    L.check(L.load().starkv_hybrid_decode(
+        ctypes.byref(lay), _ptr(q), _ptr(cache), cache.numel() * cache.element_size() // lay.page_bytes,
+        _ptr(block_table), block_table.shape[1], _ptr(seq_lens), batch, _ptr(Bk_t), _ptr(Bv),
+        _ptr(rope_table), rope_table.numel() * rope_table.element_size(), _ptr(out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
+        _stream(stream)), "starkv_hybrid_decode")
+
+
 def alloc(lay: L.Layout, num_pages: int, batch: int, max_pages: int,
           max_append_tokens: int) -> L.Sizes:
     s = L.Sizes()

@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["api.cu", "decode.cu", "store.cu", "project.cu", "append_gemv.cu", "decode_noalloc.cu",
-           "diag.cu", "absorb.cu"]
+           "diag.cu", "absorb.cu", "hybrid.cu"]
 LIB = os.path.join(HERE, "libstarkv.so")
 
 

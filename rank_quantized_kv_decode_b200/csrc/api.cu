@@ -118,16 +118,23 @@ LatDesc lat_desc(const starkv_segment& s) {
 starkv_status check_layout(const starkv_layout* lay) {
   if (!lay) return fail(STARKV_ERR_INVALID_ARG, "layout is NULL");
   starkv_layout chk;
-  const starkv_status st = starkv_layout_init(&lay->cfg, &chk);
+  const bool hybrid = lay->assignment == STARKV_ASSIGN_HYBRID;
+  if (!hybrid && lay->assignment != STARKV_ASSIGN_JOINT_KEYS)
+    return fail(STARKV_ERR_INVALID_ARG, "layout has an unknown assignment");
+  const starkv_status st =
+      hybrid ? starkv_hybrid_layout_init(&lay->hybrid, &chk) : starkv_layout_init(&lay->cfg, &chk);
   if (st != STARKV_OK) return st;
   if (std::memcmp(&chk, lay, sizeof(chk)) != 0)
-    return fail(STARKV_ERR_INVALID_ARG, "layout was not produced by starkv_layout_init for its cfg");
+    return fail(STARKV_ERR_INVALID_ARG, "layout was not produced by its layout_init for its config");
   return STARKV_OK;
 }
 
-// The formats the decode kernels implement: all four (f32, bf16, int8/int4, had43).
+// The joint-key decode calls (latent 0 the key latent, latent 1+g the value latent of KV
+// head g) take every format (f32, bf16, int8/int4, had43) but only that assignment.
 starkv_status check_decode_format(const starkv_layout* lay) {
-  (void)lay;
+  if (lay->assignment != STARKV_ASSIGN_JOINT_KEYS)
+    return fail(STARKV_ERR_UNSUPPORTED,
+                "a hybrid layout (keys head-wise, values joint) decodes with starkv_hybrid_decode");
   return STARKV_OK;
 }
 
@@ -160,14 +167,28 @@ size_t rope_bytes(const starkv_layout* lay, int max_pages) {
 int record_floats(const starkv_layout* lay) { return (2 + lay->value_rank_max + 3) / 4 * 4; }
 int tiles_for(int max_pages) { return ceil_div(max_pages * kPage, kTile); }
 
+// Hybrid decode: page ranges per sequence, so that batch x ranges is about kHybUnitsTarget.
+void hybrid_splits(int batch, int max_pages, int& nsplit, int& pps) {
+  int want = (kHybUnitsTarget + std::max(batch, 1) - 1) / std::max(batch, 1);
+  want = std::max(1, std::min(want, max_pages));
+  pps = ceil_div(max_pages, want);
+  nsplit = ceil_div(max_pages, pps);
+}
+int hybrid_rec(const starkv_layout* lay) { return (2 + lay->value_rank_total + 3) / 4 * 4; }
+
 // Bytes of the decode partial records of `batch` sequences: batch * n_q_heads * tiles * rec
-// floats, multiplied in 64 bits with an overflow check at every step.  Also refuses a
-// batch * n_q_heads above the combine kernel's grid limit (one CTA per sequence and head).
+// floats (hybrid: batch * n_q_heads * page ranges * rec), multiplied in 64 bits with an
+// overflow check at every step.  Also refuses a batch * n_q_heads above the combine kernel's
+// grid limit (one CTA per sequence and head).
 starkv_status decode_ws_bytes(const starkv_layout* lay, int32_t batch, int32_t max_pages,
                               size_t* out) {
+  const bool hybrid = lay->assignment == STARKV_ASSIGN_HYBRID;
+  int nsplit = 0, pps = 0;
+  if (hybrid) hybrid_splits(batch, max_pages, nsplit, pps);
   const uint64_t factors[4] = {static_cast<uint64_t>(lay->cfg.n_q_heads),
-                               static_cast<uint64_t>(tiles_for(max_pages)),
-                               static_cast<uint64_t>(record_floats(lay)), sizeof(float)};
+                               static_cast<uint64_t>(hybrid ? nsplit : tiles_for(max_pages)),
+                               static_cast<uint64_t>(hybrid ? hybrid_rec(lay) : record_floats(lay)),
+                               sizeof(float)};
   if (static_cast<uint64_t>(batch) * factors[0] > 0x7FFFFFFFull)
     return fail(STARKV_ERR_INVALID_ARG, "batch * n_q_heads above 2^31 - 1");
   uint64_t n = static_cast<uint64_t>(batch);
@@ -177,6 +198,59 @@ starkv_status decode_ws_bytes(const starkv_layout* lay, int32_t batch, int32_t m
     n *= f;
   }
   *out = static_cast<size_t>(n);
+  return STARKV_OK;
+}
+
+// Places latents of ``ranks`` (page order) into L.seg, sets their projection columns, the page
+// size and the stored bytes per token.  Each block starts on a 16-byte boundary.
+starkv_status place_latents(starkv_layout& L, int fmt, const int* ranks, int n) {
+  int64_t off = 0, token_bytes = 0;
+  int col = 0;
+  auto place = [&](int64_t nbytes) {
+    const int64_t o = off;
+    off = align16(off + nbytes);
+    return o;
+  };
+  for (int li = 0; li < n; ++li) {
+    const int r = ranks[li];
+    starkv_segment& s = L.seg[li];
+    s.rank = r;
+    s.col = col;
+    col += r;
+    s.off_plain = s.off_i8 = s.off_i4 = s.off_sc = -1;
+    if (fmt == STARKV_FMT_MIXED) {
+      s.n8 = (r + 3) / 4;
+      s.n4 = r - s.n8;
+      s.g8 = (s.n8 + STARKV_GROUP - 1) / STARKV_GROUP;
+      s.g4 = (s.n4 + STARKV_GROUP - 1) / STARKV_GROUP;
+      s.nb4 = (s.n4 + 1) / 2;
+      s.off_i8 = place(static_cast<int64_t>(kPage) * s.n8);
+      s.off_i4 = place(static_cast<int64_t>(kPage) * s.nb4);
+      s.off_sc = place(static_cast<int64_t>(kPage) * 2 * (s.g8 + s.g4));
+      token_bytes += s.n8 + s.nb4 + 2 * (s.g8 + s.g4);
+    } else if (fmt == STARKV_FMT_HAD43) {
+      s.n8 = (r + 4) / 5;  // the outlier block: a fifth of the channels, rounded up
+      s.n4 = r - s.n8;
+      s.g8 = (s.n8 + STARKV_GROUP - 1) / STARKV_GROUP;
+      s.g4 = (s.n4 + STARKV_GROUP - 1) / STARKV_GROUP;
+      s.pitch = (s.n8 + 1) / 2;
+      s.nb4 = 3 * ((s.n4 + 7) / 8);
+      s.off_i8 = place(static_cast<int64_t>(kPage) * s.pitch);
+      s.off_i4 = place(static_cast<int64_t>(kPage) * s.nb4);
+      s.off_sc = place(static_cast<int64_t>(kPage) * 2 * (s.g8 + s.g4));
+      token_bytes += s.pitch + s.nb4 + 2 * (s.g8 + s.g4);
+    } else {
+      const int es = elem_size(fmt);
+      s.pitch = r * es;
+      s.off_plain = place(static_cast<int64_t>(kPage) * r * es);
+      token_bytes += static_cast<int64_t>(r) * es;
+    }
+  }
+  L.n_latents = n;
+  L.proj_cols = col;
+  L.page_bytes = off;
+  L.token_bytes = token_bytes;
+  if (L.page_bytes >= (int64_t(1) << 31)) return fail(STARKV_ERR_UNSUPPORTED, "page larger than 2 GiB");
   return STARKV_OK;
 }
 
@@ -238,59 +312,79 @@ starkv_status starkv_layout_init(const starkv_config* cfg, starkv_layout* out) {
   std::memset(&L, 0, sizeof(L));
   L.cfg = c;
   for (int g = c.n_kv_heads; g < STARKV_MAX_KV_HEADS; ++g) L.cfg.value_rank[g] = 0;
-  L.n_latents = 1 + c.n_kv_heads;
-  int64_t off = 0, token_bytes = 0;
-  int col = 0, rv_total = 0, rv_max = 0;
-  auto place = [&](int64_t nbytes) {
-    const int64_t o = off;
-    off = align16(off + nbytes);
-    return o;
-  };
-  for (int li = 0; li < L.n_latents; ++li) {
-    const int r = li == 0 ? c.key_rank : c.value_rank[li - 1];
-    starkv_segment& s = L.seg[li];
-    s.rank = r;
-    s.col = col;
-    col += r;
-    if (li > 0) {
-      rv_total += r;
-      if (r > rv_max) rv_max = r;
-    }
-    s.off_plain = s.off_i8 = s.off_i4 = s.off_sc = -1;
-    if (c.fmt == STARKV_FMT_MIXED) {
-      s.n8 = (r + 3) / 4;
-      s.n4 = r - s.n8;
-      s.g8 = (s.n8 + STARKV_GROUP - 1) / STARKV_GROUP;
-      s.g4 = (s.n4 + STARKV_GROUP - 1) / STARKV_GROUP;
-      s.nb4 = (s.n4 + 1) / 2;
-      s.off_i8 = place(static_cast<int64_t>(kPage) * s.n8);
-      s.off_i4 = place(static_cast<int64_t>(kPage) * s.nb4);
-      s.off_sc = place(static_cast<int64_t>(kPage) * 2 * (s.g8 + s.g4));
-      token_bytes += s.n8 + s.nb4 + 2 * (s.g8 + s.g4);
-    } else if (c.fmt == STARKV_FMT_HAD43) {
-      s.n8 = (r + 4) / 5;  // the outlier block: a fifth of the channels, rounded up
-      s.n4 = r - s.n8;
-      s.g8 = (s.n8 + STARKV_GROUP - 1) / STARKV_GROUP;
-      s.g4 = (s.n4 + STARKV_GROUP - 1) / STARKV_GROUP;
-      s.pitch = (s.n8 + 1) / 2;
-      s.nb4 = 3 * ((s.n4 + 7) / 8);
-      s.off_i8 = place(static_cast<int64_t>(kPage) * s.pitch);
-      s.off_i4 = place(static_cast<int64_t>(kPage) * s.nb4);
-      s.off_sc = place(static_cast<int64_t>(kPage) * 2 * (s.g8 + s.g4));
-      token_bytes += s.pitch + s.nb4 + 2 * (s.g8 + s.g4);
-    } else {
-      const int es = elem_size(c.fmt);
-      s.pitch = r * es;
-      s.off_plain = place(static_cast<int64_t>(kPage) * r * es);
-      token_bytes += static_cast<int64_t>(r) * es;
-    }
+  L.assignment = STARKV_ASSIGN_JOINT_KEYS;
+  int ranks[1 + STARKV_MAX_KV_HEADS];
+  int rv_total = 0, rv_max = 0;
+  ranks[0] = c.key_rank;
+  for (int g = 0; g < c.n_kv_heads; ++g) {
+    ranks[1 + g] = c.value_rank[g];
+    rv_total += c.value_rank[g];
+    rv_max = std::max(rv_max, c.value_rank[g]);
   }
-  L.proj_cols = col;
+  const starkv_status st = place_latents(L, c.fmt, ranks, 1 + c.n_kv_heads);
+  if (st != STARKV_OK) return st;
   L.value_rank_total = rv_total;
   L.value_rank_max = rv_max;
-  L.page_bytes = off;
-  L.token_bytes = token_bytes;
-  if (L.page_bytes >= (int64_t(1) << 31)) return fail(STARKV_ERR_UNSUPPORTED, "page larger than 2 GiB");
+  *out = L;
+  return STARKV_OK;
+}
+
+starkv_status starkv_hybrid_layout_init(const starkv_hybrid_config* cfg, starkv_layout* out) {
+  if (!cfg || !out) return fail(STARKV_ERR_INVALID_ARG, "cfg/out is NULL");
+  const starkv_hybrid_config& c = *cfg;
+  if (c.n_kv_heads < 1 || c.n_kv_heads > STARKV_MAX_KV_HEADS)
+    return fail(STARKV_ERR_INVALID_ARG, "n_kv_heads must be in [1, 64]");
+  if (c.n_q_heads < c.n_kv_heads || c.n_q_heads % c.n_kv_heads != 0)
+    return fail(STARKV_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+  const int G = c.n_q_heads / c.n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(STARKV_ERR_UNSUPPORTED, "query heads per KV head must be 1, 2, 4 or 8");
+  if (c.head_dim != 64 && c.head_dim != 128)
+    return fail(STARKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (c.d_model < 16 || c.d_model % 16 != 0)
+    return fail(STARKV_ERR_INVALID_ARG, "d_model must be a positive multiple of 16");
+  for (int g = 0; g < c.n_kv_heads; ++g)
+    if (c.key_rank[g] < 16 || c.key_rank[g] % 16 != 0 || c.key_rank[g] > c.head_dim)
+      return fail(STARKV_ERR_INVALID_ARG, "key_rank[g] must be a multiple of 16 in [16, head_dim]");
+  if (c.value_rank < 16 || c.value_rank % 16 != 0 ||
+      c.value_rank > std::min(2048, c.n_kv_heads * c.head_dim))
+    return fail(STARKV_ERR_INVALID_ARG,
+                "value_rank must be a multiple of 16 in [16, min(2048, n_kv_heads * head_dim)]");
+  if (c.fmt != STARKV_FMT_F32 && c.fmt != STARKV_FMT_BF16 && c.fmt != STARKV_FMT_MIXED &&
+      c.fmt != STARKV_FMT_HAD43)
+    return fail(STARKV_ERR_INVALID_ARG, "unknown latent format");
+  if (c.page_tokens != kPage) return fail(STARKV_ERR_UNSUPPORTED, "page_tokens must be 64");
+  if (!(c.rope_theta > 1.0) || !std::isfinite(c.rope_theta))
+    return fail(STARKV_ERR_INVALID_ARG, "rope_theta must be finite and > 1");
+
+  starkv_layout L;
+  std::memset(&L, 0, sizeof(L));
+  // the shared fields; the joint-key ranks stay 0
+  L.cfg.n_q_heads = c.n_q_heads;
+  L.cfg.n_kv_heads = c.n_kv_heads;
+  L.cfg.head_dim = c.head_dim;
+  L.cfg.d_model = c.d_model;
+  L.cfg.fmt = c.fmt;
+  L.cfg.page_tokens = c.page_tokens;
+  L.cfg.rope_theta = c.rope_theta;
+  L.assignment = STARKV_ASSIGN_HYBRID;
+  // the config itself, copied field by field (no padding bytes of the caller's struct)
+  L.hybrid.n_q_heads = c.n_q_heads;
+  L.hybrid.n_kv_heads = c.n_kv_heads;
+  L.hybrid.head_dim = c.head_dim;
+  L.hybrid.d_model = c.d_model;
+  for (int g = 0; g < c.n_kv_heads; ++g) L.hybrid.key_rank[g] = c.key_rank[g];
+  L.hybrid.value_rank = c.value_rank;
+  L.hybrid.fmt = c.fmt;
+  L.hybrid.page_tokens = c.page_tokens;
+  L.hybrid.rope_theta = c.rope_theta;
+  int ranks[1 + STARKV_MAX_KV_HEADS];
+  for (int g = 0; g < c.n_kv_heads; ++g) ranks[g] = c.key_rank[g];
+  ranks[c.n_kv_heads] = c.value_rank;
+  const starkv_status st = place_latents(L, c.fmt, ranks, 1 + c.n_kv_heads);
+  if (st != STARKV_OK) return st;
+  L.value_rank_total = c.value_rank;
+  L.value_rank_max = c.value_rank;
   *out = L;
   return STARKV_OK;
 }
@@ -857,6 +951,8 @@ starkv_status starkv_absorbed_sizes(const starkv_layout* lay, int32_t batch, int
                                     int64_t* m_rows, size_t* scratch_bytes) {
   starkv_status st = check_layout(lay);
   if (st != STARKV_OK) return st;
+  st = check_decode_format(lay);
+  if (st != STARKV_OK) return st;
   if (batch < 0 || d_out < 1 || d_out > (1 << 20))
     return fail(STARKV_ERR_INVALID_ARG, "batch < 0 or d_out outside [1, 2^20]");
   if (!m_rows || !scratch_bytes) return fail(STARKV_ERR_INVALID_ARG, "NULL output pointer");
@@ -873,6 +969,8 @@ starkv_status starkv_absorb_output_weights(const starkv_layout* lay, const float
                                            const float* Wo, int32_t d_out, float* M,
                                            starkv_stream_t stream) {
   starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  st = check_decode_format(lay);
   if (st != STARKV_OK) return st;
   if (d_out < 1 || d_out > (1 << 20)) return fail(STARKV_ERR_INVALID_ARG, "d_out outside [1, 2^20]");
   if (!Bv || !Wo || !M) return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
@@ -928,6 +1026,97 @@ starkv_status starkv_decode_combine_absorbed(const starkv_layout* lay, const int
   a.batch = batch;
   e = launch_absorbed_output(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "absorbed output launch");
+  return STARKV_OK;
+}
+
+starkv_status starkv_hybrid_decode(const starkv_layout* lay, const void* q, const void* cache,
+                                   int64_t num_pages, const int32_t* block_table, int32_t max_pages,
+                                   const int32_t* seq_lens, int32_t batch, const void* Bk_t,
+                                   const float* Bv, const void* rope_table, size_t rope_table_bytes,
+                                   float* out, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_status, starkv_stream_t stream) {
+  starkv_status st = check_layout(lay);
+  if (st != STARKV_OK) return st;
+  if (lay->assignment != STARKV_ASSIGN_HYBRID)
+    return fail(STARKV_ERR_INVALID_ARG, "starkv_hybrid_decode takes a layout of starkv_hybrid_layout_init");
+  const starkv_config& c = lay->cfg;
+  if (c.fmt != STARKV_FMT_MIXED)
+    return fail(STARKV_ERR_UNSUPPORTED, "the hybrid decode kernel takes the int8/int4 format");
+  if (c.n_kv_heads > kHybMaxKv) return fail(STARKV_ERR_UNSUPPORTED, "hybrid decode: n_kv_heads > 16");
+  const int H = c.n_q_heads, rv = lay->value_rank_total;
+  const int hp = (H + 15) / 16 * 16, rvp = (rv + 63) / 64 * 64;
+  if (hp / 16 > 4 || (hp / 16) * (rvp / 64) > 8)
+    return fail(STARKV_ERR_UNSUPPORTED, "hybrid decode: ceil(H/16) * ceil(r_v/64) above 8, or H > 64");
+  if (lay->page_bytes >= (int64_t(1) << 20))
+    return fail(STARKV_ERR_UNSUPPORTED, "hybrid decode: a page of 1 MiB or more");
+  if (batch < 0 || max_pages < 1 || num_pages < 1)
+    return fail(STARKV_ERR_INVALID_ARG, "batch < 0, or max_pages/num_pages < 1");
+  if (max_pages > (1 << 24)) return fail(STARKV_ERR_INVALID_ARG, "max_pages too large");
+  if (batch == 0) return STARKV_OK;
+  if (!q || !cache || !block_table || !seq_lens || !Bk_t || !Bv || !rope_table || !out ||
+      !workspace || !dev_status)
+    return fail(STARKV_ERR_INVALID_ARG, "NULL pointer argument");
+  if ((reinterpret_cast<uintptr_t>(cache) | reinterpret_cast<uintptr_t>(Bk_t) |
+       reinterpret_cast<uintptr_t>(workspace)) & 15)
+    return fail(STARKV_ERR_INVALID_ARG, "cache, Bk_t and workspace must be 16-byte aligned");
+  if (rope_table_bytes < rope_bytes(lay, max_pages))
+    return fail(STARKV_ERR_WORKSPACE, "rope table smaller than needed for max_pages");
+  size_t ws_need = 0;
+  st = decode_ws_bytes(lay, batch, max_pages, &ws_need);
+  if (st != STARKV_OK) return st;
+  if (workspace_bytes < ws_need) return fail(STARKV_ERR_WORKSPACE, "decode workspace too small");
+  DevInfo info;
+  st = current_device(info);
+  if (st != STARKV_OK) return st;
+  HybridParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.cache = reinterpret_cast<const uint8_t*>(cache);
+  p.num_pages = num_pages;
+  p.page_bytes = static_cast<int>(lay->page_bytes);
+  p.block_table = block_table;
+  p.max_pages = max_pages;
+  p.seq_lens = seq_lens;
+  p.batch = batch;
+  p.Bk_t = reinterpret_cast<const __half*>(Bk_t);
+  p.Bv = Bv;
+  p.rope = reinterpret_cast<const float2*>(rope_table);
+  p.out = out;
+  p.ws = reinterpret_cast<float*>(workspace);
+  p.status = dev_status;
+  p.H = H;
+  p.Hkv = c.n_kv_heads;
+  p.G = H / c.n_kv_heads;
+  p.d = c.head_dim;
+  p.rv = rv;
+  p.rvp = rvp;
+  p.rec = hybrid_rec(lay);
+  hybrid_splits(batch, max_pages, p.nsplit, p.pps);
+  p.units = batch * p.nsplit;
+  p.hp = hp;
+  p.mt_pv = hp / 16;
+  p.qscale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c.head_dim)));
+  p.timeout_ns = 4000000000ull;
+  int64_t elem = 0;
+  for (int g = 0; g < c.n_kv_heads; ++g) {
+    p.key[g] = lat_desc(lay->seg[g]);
+    p.bk_elem[g] = static_cast<int>(elem);
+    elem += static_cast<int64_t>(c.head_dim) * lay->seg[g].rank;
+  }
+  p.val = lat_desc(lay->seg[c.n_kv_heads]);
+  {
+    int nq = rvp / 4;
+    for (int g = 0; g < c.n_kv_heads; ++g) nq += lay->seg[g].rank / 4;
+    p.nquad = (nq + 31) / 32 * 32;  // whole rounds of eight quads for each of four threads
+  }
+  if (!hybrid_plan(p, info.smem_optin))
+    return fail(STARKV_ERR_UNSUPPORTED, "hybrid decode: the shared-memory plan exceeds the device's limit");
+  const int grid = std::min(p.units, info.sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_hybrid_split(p, grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "hybrid split launch");
+  e = launch_hybrid_combine(p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "hybrid combine launch");
   return STARKV_OK;
 }
 

@@ -117,6 +117,44 @@ constexpr int kGemvMaxTokens = 32;
 size_t append_gemv_smem(int kslice, int n_tok);
 cudaError_t launch_append_gemv(const GemvParams& p, cudaStream_t s);
 
+// Decode with the hybrid assignment (keys head-wise, values joint).
+constexpr int kHybMaxKv = 16;       // KV heads the hybrid decode kernel takes
+constexpr int kHybUnitsTarget = 1184;  // (sequence, page range) units aimed at: 8 per SM of 148
+struct HybridParams {
+  const __nv_bfloat16* q;   // [batch][H][d]
+  const uint8_t* cache;
+  long long num_pages;
+  int page_bytes;
+  const int* block_table;   // [batch][max_pages]
+  int max_pages;
+  const int* seq_lens;
+  int batch;
+  const __half* Bk_t;       // KV head g: [d][r_k,g] at element bk_elem[g]
+  const float* Bv;          // [r_v][H_kv d]
+  const float2* rope;       // fine [128][d/2] then base [rope_tiles][d/2]
+  float* out;               // [batch][H][d]
+  float* ws;                // records [batch][nsplit][H][rec]: m (log2 units), l, a[r_v]
+  int* status;
+  int H, Hkv, G, d;
+  int rv, rvp, rec;         // joint value rank, padded to a multiple of 64, floats per record
+  int nsplit, pps, units;   // page ranges per sequence, pages per range, batch * nsplit
+  int hp, mt_pv;            // H padded to 16, its 16-row tiles
+  int nquad;                // entries of the quad table: the latents' 4-channel groups, padded
+  float qscale;             // log2(e) / sqrt(d)
+  unsigned long long timeout_ns;
+  LatDesc key[kHybMaxKv];
+  LatDesc val;
+  int bk_elem[kHybMaxKv];
+  // shared-memory plan (byte offsets), set by hybrid_plan
+  int s_bk[kHybMaxKv], s_ck[kHybMaxKv];
+  int s_cv, s_qhi, s_qlo, s_s, s_p, s_stat, s_qtab, s_page, s_bar, smem_bytes;
+};
+// Fills the shared-memory plan of ``p`` (H, Hkv, d, ranks, rvp, page_bytes set); false when
+// it exceeds ``smem_limit``.
+bool hybrid_plan(HybridParams& p, size_t smem_limit);
+cudaError_t launch_hybrid_split(const HybridParams& p, int grid, cudaStream_t s);
+cudaError_t launch_hybrid_combine(const HybridParams& p, cudaStream_t s);
+
 // Weight absorption (attention output projection folded into the value up-projection).
 struct AbsorbParams {
   const float* Bv;  // [R_v][d]

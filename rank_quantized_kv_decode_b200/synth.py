@@ -58,6 +58,47 @@ WORKLOADS = {
 }
 
 
+# The hybrid assignment (keys head-wise, values joint) at the shape of workload 4: GQA 32/8,
+# d 128, int8/int4, 32 sequences x 32768 tokens, paged.  Per-head key ranks are multiples of 16
+# (the hybrid kernel's k-step) averaging 32, the same total of 256 as workload 4's joint key;
+# one joint value latent of rank 256, the same total as workload 4's head-wise values.
+HYBRID_INDEX = 6
+HYBRID = dict(
+    name="llama3-8b-gqa-hybrid-int8int4-b32-ctx32768-paged",
+    batch=32, n_q_heads=32, n_kv_heads=8, head_dim=128, d_model=4096, context=32768,
+    spectrum_scale=256.0, key_ranks=(32, 16, 48, 32, 32, 16, 48, 32), value_rank=256,
+    fmt="mixed", rope_theta=500000.0, page_tokens=64, shuffle_pages=True,
+)
+
+
+def hybrid_workload(**overrides) -> dict:
+    """A copy of the hybrid workload with optional shape overrides."""
+    w = dict(HYBRID)
+    w.update(overrides)
+    w["index"] = HYBRID_INDEX
+    return w
+
+
+def hybrid_factors(w: dict):
+    """Factors of a hybrid layer: per KV head g, B_k,g (r_k,g x d) with orthonormal rows; the
+    joint B_v (r_v x H_kv d) with orthonormal rows.  Returned as fp64."""
+    d, Hkv = w["head_dim"], w["n_kv_heads"]
+    Bk = [haar_frame(rng(w["index"], f"Bk{g}"), d, int(r)).T for g, r in enumerate(w["key_ranks"])]
+    Bv = haar_frame(rng(w["index"], "Bv"), Hkv * d, int(w["value_rank"])).T
+    return Bk, Bv
+
+
+def hybrid_latents(w: dict, b: int, t0: int, t1: int) -> np.ndarray:
+    """fp32 latents [C_k,0 | ... | C_k,H_kv-1 | C_v] of sequence b, positions t0..t1-1, each
+    latent drawn with the spectrum's leading values as per-channel deviations."""
+    L = w["context"]
+    parts = [latent_draw(rng(w["index"], f"hk{g}:{b}"), L, spectrum(int(r), w["spectrum_scale"]))
+             for g, r in enumerate(w["key_ranks"])]
+    parts.append(latent_draw(rng(w["index"], f"hv:{b}"), L,
+                             spectrum(int(w["value_rank"]), w["spectrum_scale"])))
+    return np.concatenate(parts, axis=1)[t0:t1]
+
+
 def workload(index: int, **overrides) -> dict:
     """Return a copy of workload ``index`` with optional shape overrides (for reduced-size
     parity cases that keep the structure of the stated workload)."""

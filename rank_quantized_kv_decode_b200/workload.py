@@ -191,3 +191,56 @@ def decode(wl: Workload, **kw) -> torch.Tensor:
     api.decode_attention(wl.lay, wl.q, wl.lc.cache, wl.block_table, wl.seq_lens, wl.Bk_t, wl.Bv,
                          wl.lc.rope, wl.out, wl.lc.decode_ws, wl.lc.status, **kw)
     return wl.out
+
+
+@dataclass
+class HybridWorkload:
+    """A hybrid layer (keys head-wise, values joint) and its cache on the device."""
+
+    w: dict
+    lay: object
+    lc: api.LatentCache
+    block_table: torch.Tensor
+    seq_lens: torch.Tensor
+    q: torch.Tensor
+    Bk_t: torch.Tensor
+    Bv: torch.Tensor
+    out: torch.Tensor
+
+
+def build_hybrid(device="cuda", seq_lens=None, **overrides) -> HybridWorkload:
+    """Prepare the hybrid workload: layout, page pool, block table, queries, the factors in
+    their operand types (B_k,g^T fp16 blocks, B_v fp32) and the context latents stored with
+    starkv_quant_pack."""
+    w = synth.hybrid_workload(**overrides)
+    B, L, Hkv, d = w["batch"], w["context"], w["n_kv_heads"], w["head_dim"]
+    cfg = api.make_hybrid_config(w["n_q_heads"], Hkv, d, w["d_model"], list(w["key_ranks"]),
+                                 w["value_rank"], w["fmt"], w["rope_theta"])
+    lay = api.hybrid_layout_init(cfg)
+    max_pages = (L + 63) // 64
+    max_pages += max_pages & 1
+    lens = np.full(B, L, dtype=np.int32) if seq_lens is None else np.asarray(seq_lens, np.int32)
+    lc = api.LatentCache.create(lay, B * max_pages, B, max_pages, B, device)
+    bt = torch.from_numpy(block_table(w, max_pages)).to(device)
+    Bk, Bv = synth.hybrid_factors(w)
+    Bk_t = torch.from_numpy(np.concatenate([np.ascontiguousarray(b.T).ravel() for b in Bk])
+                            .astype(np.float32)).to(torch.float16).to(device)
+    Bv_t = torch.from_numpy(np.ascontiguousarray(Bv, dtype=np.float32)).to(device)
+    q = torch.from_numpy(queries(w)).to(torch.bfloat16).to(device)
+    out = torch.empty(B, w["n_q_heads"], d, dtype=torch.float32, device=device)
+    for b in range(B):
+        lb = int(lens[b])
+        if lb == 0:
+            continue
+        lat = torch.from_numpy(synth.hybrid_latents(w, b, 0, lb)).to(device)
+        seq = torch.full((lb,), b, dtype=torch.int32, device=device)
+        pos = torch.arange(0, lb, dtype=torch.int32, device=device)
+        api.quant_pack(lay, lat, seq, pos, bt, lc.cache, lc.status)
+    torch.cuda.synchronize(device)
+    return HybridWorkload(w, lay, lc, bt, torch.from_numpy(lens).to(device), q, Bk_t, Bv_t, out)
+
+
+def decode_hybrid(hw: HybridWorkload) -> torch.Tensor:
+    api.hybrid_decode(hw.lay, hw.q, hw.lc.cache, hw.block_table, hw.seq_lens, hw.Bk_t, hw.Bv,
+                      hw.lc.rope, hw.out, hw.lc.decode_ws, hw.lc.status)
+    return hw.out

@@ -44,7 +44,8 @@ def test_struct_sizes_match_c(lib):
     # so a ctypes struct of the wrong size would be rejected
     assert ctypes.sizeof(L.Config) == 296
     assert ctypes.sizeof(L.Segment) == 64
-    assert ctypes.sizeof(L.Layout) == 296 + 16 + 16 + 65 * 64
+    assert ctypes.sizeof(L.HybridConfig) == 296
+    assert ctypes.sizeof(L.Layout) == 296 + 16 + 16 + 65 * 64 + 8 + 296
 
 
 CASES = [
@@ -254,3 +255,110 @@ def test_binding_checks_dtype_and_size_before_the_library_sees_a_pointer(lib):
     # well-formed arguments pass the checks and stop at the device check
     with pytest.raises(ValueError, match="CUDA tensor"):
         api.decode_attention(lay, q, cache, table, seq_lens, Bk_t, Bv, cache, out, cache, i32)
+
+
+# ---- the hybrid assignment (keys head-wise, values joint)
+HYBRID_CASES = [
+    ("mixed", 32, 8, 128, 4096, [32, 16, 48, 32, 32, 16, 48, 32], 256),
+    ("mixed", 8, 2, 64, 256, [64, 16], 48),
+    ("bf16", 32, 32, 128, 4096, [16 * (1 + g % 8) for g in range(32)], 1024),
+    ("had43", 32, 8, 128, 4096, [32] * 8, 256),
+    ("f32", 4, 4, 64, 256, [16, 32, 48, 64], 128),
+]
+
+
+@pytest.mark.parametrize("fmt,H,Hkv,d,dm,kr,rv", HYBRID_CASES)
+def test_hybrid_layout_matches_oracle(lib, fmt, H, Hkv, d, dm, kr, rv):
+    lay = api.hybrid_layout_init(api.make_hybrid_config(H, Hkv, d, dm, kr, rv, fmt, 500000.0))
+    ref = O.hybrid_page_layout(fmt, kr, rv, page_tokens=64)
+    assert lay.assignment == L.ASSIGN_HYBRID
+    assert lay.page_bytes == ref["page_bytes"] and lay.token_bytes == ref["token_bytes"]
+    assert lay.n_latents == Hkv + 1
+    assert lay.proj_cols == sum(kr) + rv
+    assert lay.value_rank_total == rv and lay.value_rank_max == rv
+    assert lay.cfg.key_rank == 0 and all(lay.cfg.value_rank[g] == 0 for g in range(L.MAX_KV_HEADS))
+    assert (lay.cfg.n_q_heads, lay.cfg.n_kv_heads, lay.cfg.head_dim) == (H, Hkv, d)
+    assert [lay.hybrid.key_rank[g] for g in range(Hkv)] == kr and lay.hybrid.value_rank == rv
+    col = 0
+    for li, s in enumerate(ref["segs"]):
+        seg = lay.seg[li]
+        assert seg.rank == (kr[li] if li < Hkv else rv) == s["rank"] and seg.col == col
+        col += s["rank"]
+        if fmt == "mixed":
+            assert (seg.off_i8, seg.off_i4, seg.off_sc) == (s["i8"], s["i4"], s["sc"])
+            assert (seg.n8, seg.nb4, seg.g8, seg.g4) == (s["n8"], s["nb4"], s["g8"], s["g4"])
+        elif fmt == "had43":
+            assert (seg.off_i8, seg.off_i4, seg.off_sc) == (s["hi"], s["lo"], s["sc"])
+        else:
+            assert seg.off_plain == s["plain"] and seg.pitch == s["pitch"]
+
+
+@pytest.mark.parametrize("field,value", [("value_rank", 24), ("value_rank", 0), ("value_rank", 4096),
+                                         ("head_dim", 96), ("page_tokens", 32)])
+def test_hybrid_layout_rejects(lib, field, value):
+    cfg = api.make_hybrid_config(32, 8, 128, 4096, [32] * 8, 256, "mixed", 10000.0)
+    setattr(cfg, field, value)
+    lay = L.Layout()
+    assert lib.starkv_hybrid_layout_init(ctypes.byref(cfg), ctypes.byref(lay)) != L.OK
+
+
+@pytest.mark.parametrize("rank", [0, 8, 20, 144])
+def test_hybrid_layout_rejects_key_ranks_off_the_16_grid(lib, rank):
+    cfg = api.make_hybrid_config(32, 8, 128, 4096, [32] * 7 + [rank], 256, "mixed", 10000.0)
+    lay = L.Layout()
+    assert lib.starkv_hybrid_layout_init(ctypes.byref(cfg), ctypes.byref(lay)) == L.ERR_INVALID_ARG
+
+
+def test_hybrid_workspace_holds_one_record_per_page_range_and_head(lib):
+    lay = api.hybrid_layout_init(api.make_hybrid_config(32, 8, 128, 4096, [32] * 8, 256, "mixed",
+                                                        500000.0))
+    for batch, max_pages in [(32, 512), (1, 2048), (3, 17), (1000, 4)]:
+        s = api.alloc(lay, 10, batch, max_pages, 0)
+        want = -(-1184 // batch)
+        want = max(1, min(want, max_pages))
+        pps = -(-max_pages // want)
+        nsplit = -(-max_pages // pps)
+        assert nsplit * pps >= max_pages and (nsplit - 1) * pps < max_pages
+        rec = (2 + 256 + 3) // 4 * 4
+        assert s.decode_workspace_bytes == batch * 32 * nsplit * rec * 4
+
+
+def test_joint_key_calls_refuse_a_hybrid_layout_before_touching_the_device(lib):
+    lay = api.hybrid_layout_init(api.make_hybrid_config(32, 8, 128, 4096, [32] * 8, 256, "mixed",
+                                                        500000.0))
+    plan = L.DecodePlan()
+    assert lib.starkv_decode_plan_query(ctypes.byref(lay), 4, 16, None, 148, 232448,
+                                        ctypes.byref(plan)) == L.ERR_UNSUPPORTED
+    rows, scratch = ctypes.c_int64(0), ctypes.c_size_t(0)
+    assert lib.starkv_absorbed_sizes(ctypes.byref(lay), 4, 4096, ctypes.byref(rows),
+                                     ctypes.byref(scratch)) == L.ERR_UNSUPPORTED
+    # the decode call itself, with host dummies that it must not dereference
+    assert lib.starkv_decode_attention(ctypes.byref(lay), 16, 16, 4, 16, 16, 16, 1, 16, 16, 16,
+                                       1 << 20, 16, 16, 1 << 30, None, 16, None) == L.ERR_UNSUPPORTED
+
+
+def test_hybrid_decode_refuses_before_touching_the_device(lib):
+    joint = api.layout_init(api.make_config(32, 8, 128, 4096, 256, [32] * 8, "mixed", 500000.0))
+    args = (16, 16, 4, 16, 16, 16, 1, 16, 16, 16, 1 << 20, 16, 16, 1 << 30, 16, None)
+    assert lib.starkv_hybrid_decode(ctypes.byref(joint), *args) == L.ERR_INVALID_ARG
+    bf16 = api.hybrid_layout_init(api.make_hybrid_config(32, 8, 128, 4096, [32] * 8, 256, "bf16",
+                                                         500000.0))
+    assert lib.starkv_hybrid_decode(ctypes.byref(bf16), *args) == L.ERR_UNSUPPORTED
+    wide = api.hybrid_layout_init(api.make_hybrid_config(64, 32, 128, 4096, [32] * 32, 256,
+                                                         "mixed", 500000.0))
+    assert lib.starkv_hybrid_decode(ctypes.byref(wide), *args) == L.ERR_UNSUPPORTED  # H_kv > 16
+    big = api.hybrid_layout_init(api.make_hybrid_config(64, 8, 128, 4096, [32] * 8, 512, "mixed",
+                                                        500000.0))
+    assert lib.starkv_hybrid_decode(ctypes.byref(big), *args) == L.ERR_UNSUPPORTED  # 4 x 8 tiles
+
+
+def test_tampered_hybrid_layout_rejected(lib):
+    lay = api.hybrid_layout_init(api.make_hybrid_config(32, 8, 128, 4096, [32] * 8, 256, "mixed",
+                                                        500000.0))
+    lay.seg[8].off_sc += 16
+    s = L.Sizes()
+    assert lib.starkv_alloc(ctypes.byref(lay), 10, 1, 4, 0, ctypes.byref(s)) == L.ERR_INVALID_ARG
+    lay2 = api.hybrid_layout_init(api.make_hybrid_config(32, 8, 128, 4096, [32] * 8, 256, "mixed",
+                                                         500000.0))
+    lay2.assignment = 7
+    assert lib.starkv_alloc(ctypes.byref(lay2), 10, 1, 4, 0, ctypes.byref(s)) == L.ERR_INVALID_ARG
