@@ -41,7 +41,10 @@ MMA_DTYPE = {"f32": "tf32", "bf16": "bf16", "mixed": "f16", "had43": "f16"}
 # workload, keyed by a digest of the kernel's sources: the figure is reported only while the
 # sources are the ones it was captured with (otherwise traffic is null).
 KERNEL_SOURCES = ["decode.cu", "ptx.cuh", "internal.cuh", "api.cu"]
-SPLIT_TRAFFIC = {}  # workload index -> (source digest, bytes)
+# workload index -> (source digest, dram__bytes_read.sum + dram__bytes_write.sum of one split
+# launch): workload 4, 397396224 read + 32261888 written, captured with
+# ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum -k regex:decode_split
+SPLIT_TRAFFIC = {4: ("9eb396c1f4101960", 397396224 + 32261888)}
 
 THROTTLE_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                  0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
