@@ -37,8 +37,27 @@ int main(void) {
   int64_t rows = 0;
   size_t scratch = 0;
   if (starkv_absorbed_sizes(&lay, 2, 4096, &rows, &scratch) != STARKV_OK) return 3;
-  printf("%lld %lld %lld %d\n", (long long)lay.page_bytes, (long long)sz.cache_bytes,
-         (long long)rows, starkv_version());
+  /* the hybrid assignment: a key latent per KV head, one joint value latent */
+  starkv_hybrid_config hc;
+  memset(&hc, 0, sizeof hc);
+  hc.n_q_heads = 32;
+  hc.n_kv_heads = 8;
+  hc.head_dim = 128;
+  hc.d_model = 4096;
+  for (int g = 0; g < 8; ++g) hc.key_rank[g] = 16 * (1 + g % 3);
+  hc.value_rank = 256;
+  hc.fmt = STARKV_FMT_MIXED;
+  hc.page_tokens = 64;
+  hc.rope_theta = 500000.0;
+  starkv_layout hl;
+  if (starkv_hybrid_layout_init(&hc, &hl) != STARKV_OK) return 4;
+  if (hl.assignment != STARKV_ASSIGN_HYBRID || hl.n_latents != 9) return 5;
+  starkv_sizes hs;
+  if (starkv_alloc(&hl, 100, 2, 8, 16, &hs) != STARKV_OK) return 6;
+  /* a joint-key call refuses the hybrid layout before touching the device */
+  if (starkv_absorbed_sizes(&hl, 2, 4096, &rows, &scratch) != STARKV_ERR_UNSUPPORTED) return 7;
+  printf("%lld %lld %lld %d %d %lld\n", (long long)lay.page_bytes, (long long)sz.cache_bytes,
+         (long long)rows, starkv_version(), hl.proj_cols, (long long)hs.cache_bytes);
   return 0;
 }
 """
@@ -65,5 +84,6 @@ def test_c99_caller_compiles_links_and_runs_host_calls(tmp_path):
     if run.returncode != 0 and "error while loading shared libraries" in run.stderr:
         pytest.skip("the CUDA runtime the library links is not on the loader path here")
     assert run.returncode == 0, run.stdout + run.stderr
-    page_bytes, cache_bytes, rows, version = (int(v) for v in run.stdout.split())
+    page_bytes, cache_bytes, rows, version, hproj, hcache = (int(v) for v in run.stdout.split())
     assert cache_bytes == 100 * page_bytes and rows == 4 * 8 * 32 and version > 0
+    assert hproj == sum(16 * (1 + g % 3) for g in range(8)) + 256 and hcache % 100 == 0
