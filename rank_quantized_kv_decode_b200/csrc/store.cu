@@ -24,6 +24,7 @@ using namespace store_dev;
 // Sum of the split-K partials of one value, in split order (deterministic).  Up to 16 loads
 // are issued before the first add, so a decode step's partials arrive in one round trip.
 __device__ __forceinline__ float split_sum(const float* src, long long stride, int nsplit) {
+  if (nsplit == 1) return __ldcg(src);  // one split (a prefill-sized append): a single load
   float v = 0.f;
   for (int s0 = 0; s0 < nsplit; s0 += 16) {
     float t[16];
