@@ -502,6 +502,10 @@ __global__ void __launch_bounds__(128) hybrid_combine_kernel(const __grid_consta
   }
   const long long stride = static_cast<long long>(p.H) * p.rec;  // between page ranges
   const float* r0 = p.ws + (static_cast<long long>(b) * p.nsplit * p.H + h) * p.rec;
+  // each range's weight exp2(m_s - M) once (0 for a range without weight), in shared memory
+  // after the r_v slots of s_a when the ranges fit, else recomputed per channel
+  float* s_w = s_a + p.rv;
+  const bool wfit = p.rv + p.nsplit <= 2048;
   float M = -INFINITY;
   for (int s = 0; s < p.nsplit; ++s) {
     const float* rc = r0 + s * stride;
@@ -512,12 +516,20 @@ __global__ void __launch_bounds__(128) hybrid_combine_kernel(const __grid_consta
     const float* rc = r0 + s * stride;
     if (rc[1] > 0.f) l += rc[1] * exp2f(rc[0] - M);
   }
+  if (wfit) {
+    for (int s = tid; s < p.nsplit; s += 128) {
+      const float* rc = r0 + s * stride;
+      s_w[s] = rc[1] > 0.f ? exp2f(rc[0] - M) : 0.f;
+    }
+    __syncthreads();
+  }
   const float inv = l > 0.f ? 1.f / l : 0.f;
   for (int i = tid; i < p.rv; i += 128) {
     float a = 0.f;
     for (int s = 0; s < p.nsplit; ++s) {
       const float* rc = r0 + s * stride;
-      if (rc[1] > 0.f) a = fmaf(rc[2 + i], exp2f(rc[0] - M), a);
+      const float w = wfit ? s_w[s] : (rc[1] > 0.f ? exp2f(rc[0] - M) : 0.f);
+      if (w > 0.f) a = fmaf(rc[2 + i], w, a);
     }
     s_a[i] = a * inv;
   }
