@@ -37,19 +37,24 @@ __device__ __forceinline__ float split_sum(const float* src, long long stride, i
   return v;
 }
 
-// One warp per (token, latent, 32-channel chunk): lane = channel.  In the int8/int4 format a
-// chunk is one quantisation group (the int8 groups, then the int4 groups of the latent).
+// One warp per (token, latent, 32-channel chunk): lane = channel; token n = blockIdx.x, chunk
+// = 4 blockIdx.y + warp.  In the int8/int4 format a chunk is one quantisation group (the int8
+// groups, then the int4 groups of the latent).  FMT is the storage format.
+template <int FMT>
 __global__ void __launch_bounds__(128) store_kernel(const __grid_constant__ StoreParams p) {
   pdl_wait();
   pdl_launch_dependents();
-  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int ck = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (gw >= p.n_tok * p.chunks_per_token) return;  // whole warp
-  const int n = gw / p.chunks_per_token;
-  const ChunkLane q = chunk_lane(p, gw % p.chunks_per_token, lane);
+  if (ck >= p.chunks_per_token) return;  // whole warp
+  const int n = blockIdx.x;
+  const ChunkLane q = chunk_lane<FMT>(p, ck, lane);
   const float* src = p.src + (long long)n * p.proj_cols + p.lat[q.li].col;
   const float c = q.in ? split_sum(src + q.i, p.split_stride, p.nsplit) : 0.f;
-  store_value(p, q, n, lane, c);
+  // the page lookup flags a bad page or position once per token: in the chunk of latent 0,
+  // channel 0
+  const TokenSlot ts = locate(p, n, (q.li == 0 && q.cl == 0) ? 0 : 1, lane);
+  store_value_at<FMT>(p, q, n, lane, c, ts);
 }
 
 // One warp per (token, latent): stored value -> fp32 (scale * code for the mixed format).
@@ -116,9 +121,15 @@ __global__ void rope_init_kernel(float2* table, int half_dim, int rows, double t
 }  // namespace
 
 cudaError_t launch_store(const StoreParams& p, cudaStream_t s) {
-  const long long warps = (long long)p.n_tok * p.chunks_per_token;
-  if (warps == 0) return cudaSuccess;
-  return launch_pdl(store_kernel, dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, s, p);
+  if (p.n_tok == 0 || p.chunks_per_token == 0) return cudaSuccess;
+  const dim3 grid(static_cast<unsigned>(p.n_tok), static_cast<unsigned>((p.chunks_per_token + 3) / 4));
+  switch (p.fmt) {
+    case STARKV_FMT_F32: return launch_pdl(store_kernel<STARKV_FMT_F32>, grid, dim3(128), 0, s, p);
+    case STARKV_FMT_BF16: return launch_pdl(store_kernel<STARKV_FMT_BF16>, grid, dim3(128), 0, s, p);
+    case STARKV_FMT_MIXED: return launch_pdl(store_kernel<STARKV_FMT_MIXED>, grid, dim3(128), 0, s, p);
+    case STARKV_FMT_HAD43: return launch_pdl(store_kernel<STARKV_FMT_HAD43>, grid, dim3(128), 0, s, p);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_dequant(const StoreParams& p, cudaStream_t s) {

@@ -60,14 +60,17 @@ struct ChunkLane {
   int n4, j, i;   // channels of the second block; channel index there; channel in the latent
 };
 
+// FMT: the storage format when the caller knows it at compile time, -1 to read p.fmt.
+template <int FMT = -1>
 __device__ __forceinline__ ChunkLane chunk_lane(const StoreParams& p, int ck, int lane) {
+  const int fmt = FMT >= 0 ? FMT : p.fmt;
   ChunkLane c{};
   int li = 0;
   while (p.chunk_start[li + 1] <= ck) ++li;
   c.li = li;
   c.cl = ck - p.chunk_start[li];
   const LatDesc& d = p.lat[li];
-  c.plain = p.fmt == STARKV_FMT_F32 || p.fmt == STARKV_FMT_BF16;
+  c.plain = fmt == STARKV_FMT_F32 || fmt == STARKV_FMT_BF16;
   c.is8 = !c.plain && c.cl < d.g8;
   c.n4 = d.rank - d.n8;
   c.j = (c.plain || c.is8) ? 0 : (c.cl - d.g8) * 32 + lane;
@@ -79,8 +82,10 @@ __device__ __forceinline__ ChunkLane chunk_lane(const StoreParams& p, int ck, in
 // Store the value ``c`` of this lane's channel for token ``n`` at its page and slot ``ts``
 // (from locate; the whole warp calls it; lanes outside the chunk pass c = 0).  Writes
 // latents_out too when the caller asked for it.
+template <int FMT = -1>
 __device__ __forceinline__ void store_value_at(const StoreParams& p, const ChunkLane& q, int n,
                                                int lane, float c, const TokenSlot& ts) {
+  const int fmt = FMT >= 0 ? FMT : p.fmt;
   const LatDesc& d = p.lat[q.li];
   const int cl = q.cl, j = q.j, i = q.i, n4 = q.n4;
   const bool plain = q.plain, is8 = q.is8, in = q.in;
@@ -90,14 +95,14 @@ __device__ __forceinline__ void store_value_at(const StoreParams& p, const Chunk
   if (plain) {
     if (!in || !ts.page) return;
     uint8_t* dst = ts.page + d.off0 + ts.slot * d.pitch;
-    if (p.fmt == STARKV_FMT_F32)
+    if (fmt == STARKV_FMT_F32)
       reinterpret_cast<float*>(dst)[i] = c;
     else
       reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(c);
     return;
   }
   __half* sc = ts.page ? reinterpret_cast<__half*>(ts.page + d.off2) + ts.slot * d.ng : nullptr;
-  if (p.fmt == STARKV_FMT_HAD43) {
+  if (fmt == STARKV_FMT_HAD43) {
     const float amax = warp_max_abs(in ? fabsf(c) : 0.f);
     if (is8) {
       // 4-bit group cl: channels [32 cl, min(32 cl + 32, n8)), d.pitch packed bytes per token
@@ -150,14 +155,6 @@ __device__ __forceinline__ void store_value_at(const StoreParams& p, const Chunk
     }
     if (ts.page && lane == 0) sc[d.g8 + gi] = h;
   }
-}
-
-// The same for token ``n`` located here (the page lookup flags a bad page or position once
-// per token: in the chunk of latent 0, channel 0).
-__device__ __forceinline__ void store_value(const StoreParams& p, const ChunkLane& q, int n,
-                                            int lane, float c) {
-  const TokenSlot ts = locate(p, n, (q.li == 0 && q.cl == 0) ? 0 : 1, lane);
-  store_value_at(p, q, n, lane, c, ts);
 }
 
 }  // namespace store_dev
