@@ -282,22 +282,24 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_split_kernel(const __grid_
           __half sc[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) e[u] = tab[j0 + 4 * u];
+          // branch-free, so the eight quads' loads overlap: every quad reads two half-words
+          // at its offset (a zero quad reads the page's first bytes: its entry holds offset 0
+          // and stride 0) and its scale, and both conversions are selected by kind
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int kind = e[u].x >> 28;
-            w[u] = 0u;
-            sc[u] = __float2half_rn(0.f);
-            if (tv && kind != kQuadZero) {
-              const uint8_t* src = page + (e[u].x & 0xFFFFF) + tk * (e[u].y & 0xFFFF);
-              w[u] = kind == kQuadInt8 ? *reinterpret_cast<const uint32_t*>(src)
-                                       : static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(src));
-              sc[u] = *reinterpret_cast<const __half*>(page + e[u].z + tk * (e[u].y >> 16));
-            }
+            const uint8_t* src = page + (e[u].x & 0xFFFFF) + tk * (e[u].y & 0xFFFF);
+            const uint32_t lo = *reinterpret_cast<const unsigned short*>(src);
+            const uint32_t hi = *reinterpret_cast<const unsigned short*>(src + 2);
+            w[u] = (e[u].x >> 28) == kQuadInt8 ? (lo | (hi << 16)) : lo;
+            sc[u] = *reinterpret_cast<const __half*>(page + e[u].z + tk * (e[u].y >> 16));
           }
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int kind = e[u].x >> 28;
-            const uint2 v = (tv && kind != kQuadZero) ? dequant_codes(w[u], kind, sc[u]) : make_uint2(0u, 0u);
+            const uint2 v8 = dequant_codes(w[u], kQuadInt8, sc[u]);
+            const uint2 v4 = dequant_codes(w[u], kQuadInt4, sc[u]);
+            uint2 v = kind == kQuadInt8 ? v8 : v4;
+            if (!tv || kind == kQuadZero) v = make_uint2(0u, 0u);
             *reinterpret_cast<uint2*>(smem + (e[u].w & 0xFFFFF) + tk * ((e[u].w >> 20) << 4)) = v;
           }
         }
