@@ -364,7 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_split_kernel(const __grid_
           const int hq = gid < p.G ? g * p.G + gid : p.H;
           const uint32_t qh = smem_u32(sQhi + hq * QP) + 4 * tig;
           const uint32_t ql = smem_u32(sQlo + hq * QP) + 4 * tig;
-          float sc[4] = {0.f, 0.f, 0.f, 0.f};
+          // six independent accumulators (the three products x the parity of the k-step), so
+          // consecutive MMAs do not wait on one another; added in a fixed order at the end
+          float sp[6][4];
+#pragma unroll
+          for (int i = 0; i < 6; ++i) sp[i][0] = sp[i][1] = sp[i][2] = sp[i][3] = 0.f;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             uint32_t ah[4], al[4];
@@ -374,10 +378,15 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_split_kernel(const __grid_
             split_h2(k[2 * kk + 1][2], k[2 * kk + 1][3], ah[3], al[3]);
             const uint32_t bh0 = ld_shared_u32(qh + kk * 32), bh1 = ld_shared_u32(qh + kk * 32 + 16);
             const uint32_t bl0 = ld_shared_u32(ql + kk * 32), bl1 = ld_shared_u32(ql + kk * 32 + 16);
-            mma_f16(sc, ah[0], ah[1], ah[2], ah[3], bh0, bh1);
-            mma_f16(sc, al[0], al[1], al[2], al[3], bh0, bh1);
-            mma_f16(sc, ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+            const int o = 3 * (kk & 1);
+            mma_f16(sp[o], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+            mma_f16(sp[o + 1], al[0], al[1], al[2], al[3], bh0, bh1);
+            mma_f16(sp[o + 2], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
           }
+          float sc[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            sc[e] = ((sp[0][e] + sp[3][e]) + (sp[1][e] + sp[4][e])) + (sp[2][e] + sp[5][e]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int hh = 2 * tig + (e & 1);
